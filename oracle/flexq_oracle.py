@@ -1,0 +1,235 @@
+"""CPU oracle for FlexQ's group-quantized W6A6 / W6A8 linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may call it.  It shares no code, table or constant generator with
+the CUDA library; it is a slow, literal restatement of what the method
+computes, written so that each step can be checked against the method's
+description by eye.
+
+What the method computes (FlexQ: Efficient Post-training INT6 Quantization
+for LLM Serving via Algorithm-System Co-Design):
+
+* Weights are quantized uniformly to 6 bits in every layer (arXiv abstract);
+  activations to 6 bits, or to 8 bits in sensitive layers (abstract; drgamma
+  blog, "Fine-Grained Quantization and Layer Sensitivity").
+* Both operands use fine-grained group quantization: values are split into
+  small groups that share one scale (blog, "Fine-Grained Quantization and
+  Layer Sensitivity"), and the groups run along the K dimension (blog,
+  "Bridging Software and Hardware with BTC").
+* The product is a sum of integer products that is recombined with the
+  scales, with dequantization fused into the GEMM (blog, "Bridging Software
+  and Hardware with BTC").  Per K-group g this is the exact integer partial
+  P_g[m, n] = sum_{k in g} qa[m, k] * qw[n, k], and the output is
+  Y[m, n] = sum_g P_g[m, n] * sa[m, g] * sw[n, g].
+
+Readings where the pages are silent (each listed in the design notes):
+
+* symmetric codes, no zero point; code range [-Q, Q] with Q = 31 for 6 bits
+  and Q = 127 for 8 bits, scale = absmax / Q;
+* the scale is computed in FP32 (IEEE division), stored as FP16
+  (round-to-nearest-even), and the codes divide by the *stored* FP16 scale
+  (IEEE FP32 division), round half to even, then clamp to [-Q, Q];
+* a group whose FP16 scale is zero (all-zero, or underflowing) has scale 0
+  and all codes 0;
+* the 6-bit weight container packs 4 codes into 3 bytes, little endian,
+  code i in bits [6i, 6i+6) as 6-bit two's complement ("canonical form");
+  the device form is a fixed permutation of those bytes into 128-row tiles
+  (``reorder_to_device_form``);
+* Y is formed in FP64 from the exact integer partials and the exact FP16
+  scales, then rounded once to FP16 (round-to-nearest-even).
+
+The FP16 codec is numpy's float16 conversion (a library primitive); the tests
+pin it against torch's independent converter and against the round-to-
+nearest-even definition at every midpoint between adjacent FP16 values.
+"""
+
+import numpy as np
+
+Q_WEIGHT = 31
+Q_ACT = {6: 31, 8: 127}
+
+
+# --------------------------------------------------------------------------
+# group quantization (weights: rows = output channels n; activations: rows =
+# tokens m; groups of ``gs`` consecutive k within a row)
+# --------------------------------------------------------------------------
+def quantize_groups(x16, gs, qmax):
+    """Symmetric per-group quantization of an FP16 matrix.
+
+    x16  : float16 array [R, K]; K % gs == 0; all values finite.
+    gs   : group size along K.
+    qmax : largest code magnitude Q (31 for 6-bit, 127 for 8-bit).
+    Returns (codes int8 [R, K], scales float16 [R, K // gs]).
+
+    Per group: amax = max |x| (exact in FP32); s = fp16_rne(amax / Q) with an
+    IEEE FP32 division; code = clamp(rint_half_even(x / s), -Q, Q) with an IEEE
+    FP32 division by the stored FP16 scale; a zero scale gives zero codes.
+    """
+    x16 = np.asarray(x16, dtype=np.float16)
+    R, K = x16.shape
+    assert K % gs == 0, "K must be a multiple of the group size"
+    G = K // gs
+    x32 = x16.astype(np.float32).reshape(R, G, gs)          # exact widening
+    assert np.all(np.isfinite(x32)), "non-finite inputs are out of contract"
+    amax = np.abs(x32).max(axis=2)                           # exact
+    s32 = amax / np.float32(qmax)                            # IEEE fp32 divide
+    assert s32.dtype == np.float32
+    s16 = s32.astype(np.float16)                             # RNE to fp16
+    s16_as_f32 = s16.astype(np.float32)                      # exact widening
+    zero = s16_as_f32 == 0
+    safe = np.where(zero, np.float32(1), s16_as_f32)
+    ratio = x32 / safe[:, :, None]                           # IEEE fp32 divide
+    assert ratio.dtype == np.float32
+    q = np.rint(ratio)                                       # half to even
+    q = np.clip(q, -qmax, qmax)
+    q = np.where(zero[:, :, None], np.float32(0), q)
+    return q.astype(np.int8).reshape(R, K), s16
+
+
+def quantize_weight(w16, gs):
+    """6-bit weight quantization: codes in [-31, 31], FP16 scales [N, K/gs]."""
+    return quantize_groups(w16, gs, Q_WEIGHT)
+
+
+def quantize_act(x16, gs, bits):
+    """6- or 8-bit activation quantization: codes in [-Q, Q], scales [M, K/gs]."""
+    return quantize_groups(x16, gs, Q_ACT[bits])
+
+
+def dequantize(codes, scales, gs):
+    """codes * scale per group, in FP64 (exact: code and FP16 scale products
+    need at most 18 significant bits)."""
+    R, K = codes.shape
+    s = np.repeat(scales.astype(np.float64), gs, axis=1)
+    return codes.astype(np.float64) * s
+
+
+# --------------------------------------------------------------------------
+# 6-bit container: canonical packing (4 codes -> 3 bytes)
+# --------------------------------------------------------------------------
+def pack_canonical(codes):
+    """Pack int8 codes in [-32, 31] of shape [N, K] (K % 4 == 0) into uint8
+    [N, 3K/4].  For codes c0..c3 at k = 4j..4j+3 with u_i = c_i & 0x3F, the
+    24-bit word u0 | u1<<6 | u2<<12 | u3<<18 is stored little endian at bytes
+    3j, 3j+1, 3j+2."""
+    codes = np.asarray(codes)
+    N, K = codes.shape
+    assert K % 4 == 0
+    assert codes.min(initial=0) >= -32 and codes.max(initial=0) <= 31
+    u = (codes.astype(np.int32) & 0x3F).astype(np.uint32).reshape(N, K // 4, 4)
+    word = u[..., 0] | (u[..., 1] << 6) | (u[..., 2] << 12) | (u[..., 3] << 18)
+    out = np.empty((N, K // 4, 3), dtype=np.uint8)
+    out[..., 0] = word & 0xFF
+    out[..., 1] = (word >> 8) & 0xFF
+    out[..., 2] = (word >> 16) & 0xFF
+    return out.reshape(N, 3 * K // 4)
+
+
+def unpack_canonical(packed, K):
+    """Inverse of pack_canonical: uint8 [N, 3K/4] -> int8 codes [N, K]."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    N = packed.shape[0]
+    b = packed.reshape(N, K // 4, 3).astype(np.uint32)
+    word = b[..., 0] | (b[..., 1] << 8) | (b[..., 2] << 16)
+    fields = np.stack([(word >> (6 * i)) & 0x3F for i in range(4)], axis=-1)
+    signed = fields.astype(np.int32) - 64 * (fields >= 32)
+    return signed.reshape(N, K).astype(np.int8)
+
+
+# --------------------------------------------------------------------------
+# device form: canonical bytes permuted into 128-row x 128-k tiles
+# --------------------------------------------------------------------------
+TILE_ROWS = 128          # weight rows per tile
+TILE_K = 128             # codes per row per tile (96 packed bytes)
+CHUNK = 16               # bytes per chunk; 6 chunks per row per tile
+
+
+def reorder_to_device_form(packed, N, K):
+    """Permute canonical packed bytes [N, 3K/4] into the device form.
+
+    The device form is a flat byte array of (N/128) * (K/128) tiles of 12288
+    bytes; tile (nt, kb) holds rows nt*128 .. nt*128+127 and codes
+    kb*128 .. kb*128+127.  Inside a tile the 96 bytes of each row are cut into
+    six 16-byte chunks and stored chunk-major: byte b of chunk j of row r sits
+    at offset (j*128 + r)*16 + b.  In other words, device byte
+    [nt][kb][j][r][b] = canonical byte [nt*128 + r][kb*96 + 16*j + b].
+    """
+    assert N % TILE_ROWS == 0 and K % TILE_K == 0
+    NT, KB = N // TILE_ROWS, K // TILE_K
+    v = np.asarray(packed, dtype=np.uint8).reshape(NT, TILE_ROWS, KB, 6, CHUNK)
+    return np.ascontiguousarray(v.transpose(0, 2, 3, 1, 4)).reshape(-1)
+
+
+def device_form_to_canonical(dev, N, K):
+    """Inverse permutation of reorder_to_device_form."""
+    NT, KB = N // TILE_ROWS, K // TILE_K
+    v = np.asarray(dev, dtype=np.uint8).reshape(NT, KB, 6, TILE_ROWS, CHUNK)
+    return np.ascontiguousarray(v.transpose(0, 3, 1, 2, 4)).reshape(N, 3 * K // 4)
+
+
+# --------------------------------------------------------------------------
+# the GEMM: exact per-group integer partials, FP64 rescale, one FP16 rounding
+# --------------------------------------------------------------------------
+def group_partials(qa, qw, gs):
+    """P[g, m, n] = sum_{k in group g} qa[m, k] * qw[n, k], in int64.
+
+    qa: int codes [M, K]; qw: int codes [N, K].  Asserts that every partial
+    fits in int32 (the device accumulates each group exactly in int32)."""
+    qa = np.asarray(qa).astype(np.int64)
+    qw = np.asarray(qw).astype(np.int64)
+    M, K = qa.shape
+    N = qw.shape[0]
+    assert qw.shape[1] == K and K % gs == 0
+    G = K // gs
+    P = np.empty((G, M, N), dtype=np.int64)
+    for g in range(G):
+        ks = slice(g * gs, (g + 1) * gs)
+        P[g] = qa[:, ks] @ qw[:, ks].T
+    assert np.abs(P).max(initial=0) < 2**31
+    return P
+
+
+def rescale_fp64(P, sa, sw):
+    """Y64[m, n] = sum_g P[g, m, n] * sa[m, g] * sw[n, g] in FP64.
+
+    For codes the quantizers produce (|P| < 2^21) each term is exact in FP64
+    (P times two 11-bit FP16 significands); only the sum over groups rounds,
+    at FP64 precision."""
+    G, M, N = P.shape
+    sa64 = np.asarray(sa).astype(np.float64)    # [M, G], exact widening
+    sw64 = np.asarray(sw).astype(np.float64)    # [N, G]
+    Y = np.zeros((M, N), dtype=np.float64)
+    for g in range(G):
+        Y += P[g].astype(np.float64) * sa64[:, g][:, None] * sw64[:, g][None, :]
+    return Y
+
+
+def gemm_fp64(qa, sa, qw, sw, gs):
+    """Y64 for codes + scales of both operands."""
+    return rescale_fp64(group_partials(qa, qw, gs), sa, sw)
+
+
+def to_fp16(y64):
+    """Round FP64 values once to FP16 (round to nearest even, overflow to inf)."""
+    return np.asarray(y64, dtype=np.float64).astype(np.float16)
+
+
+def linear_layer(x16, w16, gs, act_bits):
+    """The whole layer on FP16 inputs: quantize both operands, form Y64 and
+    its FP16 rounding.  Returns a dict of every intermediate."""
+    qw, sw = quantize_weight(w16, gs)
+    qa, sa = quantize_act(x16, gs, act_bits)
+    P = group_partials(qa, qw, gs)
+    y64 = rescale_fp64(P, sa, sw)
+    return {"qw": qw, "sw": sw, "qa": qa, "sa": sa, "P": P, "y64": y64,
+            "y16": to_fp16(y64)}
+
+
+def rel_err_vs_max(y_test, y_ref):
+    """max |y_test - y_ref| / max |y_ref| (the output tolerance measure)."""
+    y_test = np.asarray(y_test, dtype=np.float64)
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    denom = np.abs(y_ref).max(initial=0.0)
+    diff = np.abs(y_test - y_ref).max(initial=0.0)
+    return diff / denom if denom > 0 else diff
