@@ -1,0 +1,434 @@
+// flexq_api.cu -- host side of the C ABI declared in include/flexq.h:
+// argument validation, launch planning, tensor-map encoding, kernel launches
+// and the device status word.  Every kernel lives in this translation unit
+// so that they share the status word without relocatable device code.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/flexq.h"
+#include "flexq_gemm.cuh"
+#include "flexq_quant.cuh"
+
+namespace {
+
+// Status word written by kernels: [0] code, [1] where, [2] block, [3] unused.
+__device__ unsigned int g_flexq_status[4];
+
+thread_local std::string t_last_error;
+
+int fail(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return status;
+}
+
+int ok() {
+  t_last_error.clear();
+  return FLEXQ_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(FLEXQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+bool valid_gs(int gs) { return gs == 32 || gs == 64 || gs == 128 || gs == 256; }
+
+std::atomic<int> g_force_tokens{0};
+std::atomic<int> g_force_split{0};
+std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+std::atomic<int> g_inject_stall{0};
+
+// ---------------------------------------------------------- device state --
+constexpr int kMaxDevices = 64;
+struct DeviceState {
+  bool ready = false;
+  int sms = 148;
+  unsigned int* status = nullptr;
+  unsigned attr_mask = 0;        // which GEMM instantiations got their smem limit
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+int device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FLEXQ_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_flexq_status);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+    st.sms = sms;
+    st.status = static_cast<unsigned int*>(p);
+    st.ready = true;
+  }
+  *out = &st;
+  return FLEXQ_OK;
+}
+
+int sm_count_or_default() {
+  int n = 0;
+  if (cudaGetDeviceCount(&n) != cudaSuccess || n == 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 148;
+  }
+  return sms;
+}
+
+// ------------------------------------------------------------ validation --
+int check_gemm_shape(int M, int N, int K, int gs) {
+  if (M < 0 || N <= 0 || K <= 0)
+    return fail(FLEXQ_ERR_INVALID_ARG, "sizes must be M >= 0, N > 0, K > 0 (M=%d N=%d K=%d)", M, N, K);
+  if (!valid_gs(gs)) return fail(FLEXQ_ERR_UNSUPPORTED, "group_size %d not in {32,64,128,256}", gs);
+  if (N % 128) return fail(FLEXQ_ERR_UNSUPPORTED, "N=%d is not a multiple of 128", N);
+  if (K % 128) return fail(FLEXQ_ERR_UNSUPPORTED, "K=%d is not a multiple of 128", K);
+  if (K % gs) return fail(FLEXQ_ERR_UNSUPPORTED, "K=%d is not a multiple of group_size %d", K, gs);
+  if (N / 128 > 65535) return fail(FLEXQ_ERR_UNSUPPORTED, "N=%d too large", N);
+  return FLEXQ_OK;
+}
+
+int check_ptrs(int n, const void* const* ptrs, const char* const* names) {
+  for (int i = 0; i < n; ++i) {
+    if (!ptrs[i]) return fail(FLEXQ_ERR_INVALID_ARG, "%s is NULL", names[i]);
+    if (!aligned16(ptrs[i])) return fail(FLEXQ_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+  }
+  return FLEXQ_OK;
+}
+
+// --------------------------------------------------------------- planning --
+int max_split_for(int T) {
+  switch (T) {
+    case 16: return flexq::GemmCfg<16>::kMaxSplit;
+    case 32: return flexq::GemmCfg<32>::kMaxSplit;
+    case 64: return flexq::GemmCfg<64>::kMaxSplit;
+    default: return flexq::GemmCfg<128>::kMaxSplit;
+  }
+}
+
+struct Plan {
+  int T;
+  int split;
+  long long ctas;
+};
+
+Plan make_plan(int M, int N, int K, int gs, int sms, bool partials) {
+  Plan p;
+  const int units = (K / 128) / (gs > 128 ? gs / 128 : 1);
+  p.T = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  const long long tiles = static_cast<long long>(N / 128) * ((M + p.T - 1) / p.T);
+  const long long slots = static_cast<long long>(sms) * (p.T <= 64 ? 2 : 1);
+  long long s = (slots + tiles / 2) / tiles;          // round(slots / tiles)
+  if (s < 1) s = 1;
+  if (s > max_split_for(p.T)) s = max_split_for(p.T);
+  if (s > units) s = units;
+  p.split = static_cast<int>(s);
+  const int fT = g_force_tokens.load(), fS = g_force_split.load();
+  if (fT == 16 || fT == 32 || fT == 64 || fT == 128) {
+    if (fT >= p.T || fT >= M) p.T = fT;      // a tile must cover >= 1 token row
+    if (p.split > max_split_for(p.T)) p.split = max_split_for(p.T);
+  }
+  if (fS >= 1 && fS <= max_split_for(p.T) && fS <= units) p.split = fS;
+  if (partials) p.split = 1;
+  p.ctas = static_cast<long long>(p.split) * (N / 128) * ((M + p.T - 1) / p.T);
+  return p;
+}
+
+// ------------------------------------------------------------ tensor map --
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// int8 activations [M, K] row-major; box = 128 bytes x T rows, 128-byte
+// swizzle; rows past M read as zero.
+int encode_x_map(CUtensorMap* map, const void* xq, int M, int K, int T) {
+  auto fn = encode_fn();
+  if (!fn) return fail(FLEXQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(T)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(xq), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FLEXQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return FLEXQ_OK;
+}
+
+// --------------------------------------------------------------- launches --
+template <int T>
+int ctrl_offset_for(int split) {
+  using Cfg = flexq::GemmCfg<T>;
+  int stage = Cfg::kStages * Cfg::kStageBytes;
+  int red = (split - 1) * 128 * T * 4;
+  int off = stage > red ? stage : red;
+  return (off + 15) & ~15;
+}
+
+template <int T>
+int smem_bytes_for(int split) {
+  return 1024 + ctrl_offset_for<T>(split) + static_cast<int>(sizeof(flexq::GemmCtrl<T>));
+}
+
+template <int T, bool PARTIALS>
+int launch_gemm_t(DeviceState* st, const CUtensorMap& map, flexq::GemmArgs a, cudaStream_t stream) {
+  using Cfg = flexq::GemmCfg<T>;
+  auto kern = flexq::gemm_w6ax_kernel<T, PARTIALS>;
+  const unsigned bit = 1u << ((T == 16 ? 0 : T == 32 ? 1 : T == 64 ? 2 : 3) + (PARTIALS ? 4 : 0));
+  {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!(st->attr_mask & bit)) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           smem_bytes_for<T>(Cfg::kMaxSplit));
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+      st->attr_mask |= bit;
+    }
+  }
+  a.ctrl_offset = ctrl_offset_for<T>(a.split);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.split), static_cast<unsigned>(a.N / 128),
+                     static_cast<unsigned>((a.M + T - 1) / T));
+  cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes_for<T>(a.split));
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(a.split);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.split > 1 ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map, a);
+  if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
+  return FLEXQ_OK;
+}
+
+int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, const void* Wp,
+                const void* Ws, void* Y, int32_t* P, bool partials, void* stream) {
+  int rc = check_gemm_shape(M, N, K, gs);
+  if (rc) return rc;
+  if (partials) {
+    const void* ptrs[] = {Xq, Wp, P};
+    const char* names[] = {"Xq", "Wq_packed", "P"};
+    if ((rc = check_ptrs(3, ptrs, names))) return rc;
+  } else {
+    const void* ptrs[] = {Xq, Xs, Wp, Ws, Y};
+    const char* names[] = {"Xq", "X_scales", "Wq_packed", "W_scales", "Y"};
+    if ((rc = check_ptrs(5, ptrs, names))) return rc;
+  }
+  if (M == 0) return ok();
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  const Plan plan = make_plan(M, N, K, gs, st->sms, partials);
+  CUtensorMap map;
+  if ((rc = encode_x_map(&map, Xq, M, K, plan.T))) return rc;
+  flexq::GemmArgs a = {};
+  a.xs = static_cast<const __half*>(Xs);
+  a.wp = static_cast<const uint8_t*>(Wp);
+  a.ws = static_cast<const __half*>(Ws);
+  a.y = static_cast<__half*>(Y);
+  a.p = P;
+  a.status = st->status;
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  a.M = M; a.N = N; a.K = K; a.gs = gs; a.split = plan.split;
+  a.stall = g_inject_stall.exchange(0);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (plan.T) {
+    case 16: rc = partials ? launch_gemm_t<16, true>(st, map, a, s) : launch_gemm_t<16, false>(st, map, a, s); break;
+    case 32: rc = partials ? launch_gemm_t<32, true>(st, map, a, s) : launch_gemm_t<32, false>(st, map, a, s); break;
+    case 64: rc = partials ? launch_gemm_t<64, true>(st, map, a, s) : launch_gemm_t<64, false>(st, map, a, s); break;
+    default: rc = partials ? launch_gemm_t<128, true>(st, map, a, s) : launch_gemm_t<128, false>(st, map, a, s); break;
+  }
+  return rc ? rc : ok();
+}
+
+}  // namespace
+
+// ===================================================================== ABI ==
+extern "C" {
+
+const char* flexq_status_string(int status) {
+  switch (status) {
+    case FLEXQ_OK: return "FLEXQ_OK";
+    case FLEXQ_ERR_INVALID_ARG: return "FLEXQ_ERR_INVALID_ARG";
+    case FLEXQ_ERR_UNSUPPORTED: return "FLEXQ_ERR_UNSUPPORTED";
+    case FLEXQ_ERR_MISALIGNED: return "FLEXQ_ERR_MISALIGNED";
+    case FLEXQ_ERR_CUDA: return "FLEXQ_ERR_CUDA";
+    case FLEXQ_ERR_DEVICE_TIMEOUT: return "FLEXQ_ERR_DEVICE_TIMEOUT";
+    default: return "FLEXQ_ERR_UNKNOWN";
+  }
+}
+
+const char* flexq_last_error_message(void) { return t_last_error.c_str(); }
+
+size_t flexq_weight_packed_bytes(int N, int K, int group_size) {
+  if (N <= 0 || K <= 0 || N % 128 || K % 128 || !valid_gs(group_size) || K % group_size) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(K) / 4 * 3;
+}
+
+int flexq_quantize_weight(int N, int K, int group_size, const void* W_fp16, void* Wq_packed,
+                          void* W_scales_fp16, void* stream) {
+  int rc = check_gemm_shape(1, N, K, group_size);
+  if (rc) return rc;
+  const void* ptrs[] = {W_fp16, Wq_packed, W_scales_fp16};
+  const char* names[] = {"W_fp16", "Wq_packed", "W_scales_fp16"};
+  if ((rc = check_ptrs(3, ptrs, names))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long G = K / group_size;
+  const long long n1 = static_cast<long long>(N) * G;
+  flexq::weight_scale_kernel<<<static_cast<unsigned>((n1 + 255) / 256), 256, 0, s>>>(
+      static_cast<const __half*>(W_fp16), static_cast<__half*>(W_scales_fp16), N, K, group_size);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "weight_scale_kernel launch");
+  const long long n2 = static_cast<long long>(N) * (K / 128) * 2;
+  flexq::weight_pack_kernel<<<static_cast<unsigned>((n2 + 255) / 256), 256, 0, s>>>(
+      static_cast<const __half*>(W_fp16), static_cast<const __half*>(W_scales_fp16),
+      static_cast<uint8_t*>(Wq_packed), N, K, group_size);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "weight_pack_kernel launch");
+  return ok();
+}
+
+int flexq_quantize_act(int M, int K, int group_size, int bits, const void* X_fp16, int8_t* Xq,
+                       void* X_scales_fp16, void* stream) {
+  if (M < 0 || K <= 0) return fail(FLEXQ_ERR_INVALID_ARG, "sizes must be M >= 0, K > 0 (M=%d K=%d)", M, K);
+  if (bits != 6 && bits != 8) return fail(FLEXQ_ERR_INVALID_ARG, "bits=%d is not 6 or 8", bits);
+  if (!valid_gs(group_size)) return fail(FLEXQ_ERR_UNSUPPORTED, "group_size %d not in {32,64,128,256}", group_size);
+  if (K % group_size) return fail(FLEXQ_ERR_UNSUPPORTED, "K=%d is not a multiple of group_size %d", K, group_size);
+  const void* ptrs[] = {X_fp16, Xq, X_scales_fp16};
+  const char* names[] = {"X_fp16", "Xq", "X_scales_fp16"};
+  int rc = check_ptrs(3, ptrs, names);
+  if (rc) return rc;
+  if (M == 0) return ok();
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  const long long chunks = static_cast<long long>(M) * K / 8;
+  long long blocks = (chunks + 255) / 256;
+  const long long cap = static_cast<long long>(st->sms) * 16;
+  if (blocks > cap) blocks = cap;
+  const int qmax = bits == 6 ? 31 : 127;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint4* x = static_cast<const uint4*>(X_fp16);
+  uint2* q = reinterpret_cast<uint2*>(Xq);
+  __half* xs = static_cast<__half*>(X_scales_fp16);
+  const int cpr = K / 8;
+  switch (group_size) {
+    case 32: flexq::quant_act_kernel<32><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, qmax); break;
+    case 64: flexq::quant_act_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, qmax); break;
+    case 128: flexq::quant_act_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, qmax); break;
+    default: flexq::quant_act_kernel<256><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, qmax); break;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "quant_act_kernel launch");
+  return ok();
+}
+
+int flexq_gemm_w6a6(int M, int N, int K, int group_size, const int8_t* Xq, const void* X_scales,
+                    const void* Wq_packed, const void* W_scales, void* Y_fp16, void* stream) {
+  return gemm_common(M, N, K, group_size, Xq, X_scales, Wq_packed, W_scales, Y_fp16, nullptr,
+                     false, stream);
+}
+
+int flexq_gemm_w6a8(int M, int N, int K, int group_size, const int8_t* Xq, const void* X_scales,
+                    const void* Wq_packed, const void* W_scales, void* Y_fp16, void* stream) {
+  return gemm_common(M, N, K, group_size, Xq, X_scales, Wq_packed, W_scales, Y_fp16, nullptr,
+                     false, stream);
+}
+
+int flexq_debug_group_partials(int M, int N, int K, int group_size, const int8_t* Xq,
+                               const void* Wq_packed, int32_t* P, void* stream) {
+  return gemm_common(M, N, K, group_size, Xq, nullptr, Wq_packed, nullptr, nullptr, P, true,
+                     stream);
+}
+
+int flexq_gemm_plan(int M, int N, int K, int group_size, int* tile_tokens, int* k_split,
+                    int* ctas) {
+  int rc = check_gemm_shape(M, N, K, group_size);
+  if (rc) return rc;
+  if (M == 0) {
+    if (tile_tokens) *tile_tokens = 0;
+    if (k_split) *k_split = 0;
+    if (ctas) *ctas = 0;
+    return ok();
+  }
+  const Plan p = make_plan(M, N, K, group_size, sm_count_or_default(), false);
+  if (tile_tokens) *tile_tokens = p.T;
+  if (k_split) *k_split = p.split;
+  if (ctas) *ctas = static_cast<int>(p.ctas);
+  return ok();
+}
+
+int flexq_debug_force_plan(int tile_tokens, int k_split) {
+  if (!(tile_tokens == 0 || tile_tokens == 16 || tile_tokens == 32 || tile_tokens == 64 ||
+        tile_tokens == 128))
+    return fail(FLEXQ_ERR_INVALID_ARG, "tile_tokens %d not in {0,16,32,64,128}", tile_tokens);
+  if (k_split < 0 || k_split > 8) return fail(FLEXQ_ERR_INVALID_ARG, "k_split %d not in 0..8", k_split);
+  g_force_tokens.store(tile_tokens);
+  g_force_split.store(k_split);
+  return ok();
+}
+
+int flexq_set_wait_limit_ns(uint64_t limit_ns) {
+  if (limit_ns == 0) return fail(FLEXQ_ERR_INVALID_ARG, "wait limit must be > 0");
+  g_wait_limit_ns.store(limit_ns);
+  return ok();
+}
+
+int flexq_debug_inject_stall(int enable) {
+  g_inject_stall.store(enable ? 1 : 0);
+  return ok();
+}
+
+int flexq_get_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc) return rc;
+  unsigned int h[4] = {0, 0, 0, 0};
+  e = cudaMemcpy(h, st->status, sizeof(h), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  if (h[0] == 0) return ok();
+  e = cudaMemset(st->status, 0, sizeof(h));
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+  static const char* roles[] = {"producer", "mma", "unpack(full)", "unpack(a_empty)", "epilogue"};
+  return fail(static_cast<int>(h[0]), "device wait timed out in the %s role of block %u",
+              h[1] < 5 ? roles[h[1]] : "?", h[2]);
+}
+
+}  // extern "C"

@@ -1,0 +1,443 @@
+// flexq_gemm.cuh -- the W6A6 / W6A8 group GEMM on tcgen05 tensor cores.
+//
+// What it computes (FlexQ paper, arXiv abstract; drgamma blog, "Bridging
+// Software and Hardware with BTC"): for every K-group g the exact integer
+// partial P_g[m,n] = sum_{k in g} qa[m,k] * qw[n,k], recombined with the
+// group scales, Y[m,n] = sum_g P_g[m,n] * sa[m,g] * sw[n,g], dequantization
+// fused into the GEMM.  The pages' kernel decomposes 6-bit operands into
+// 1-bit planes for binary tensor cores; on sm_100a one exact int8 MMA
+// replaces all plane products, so here the 6-bit weight codes are unpacked
+// losslessly to int8 and multiplied with tcgen05.mma.kind::i8.
+//
+// Orientation ("swap AB"): the MMA's M side is 128 weight rows, its N side
+// is T tokens.  Per CTA: one 128-row weight tile, one T-token tile and a
+// contiguous, group-aligned range of K (a cluster of `split` CTAs shares the
+// output tile and reduces through distributed shared memory).
+//
+// Warp roles (all pipeline waits are bounded, see mbar_wait):
+//   warp 0      producer: TMA tile of the int8 activations (T rows x 128 B,
+//               128-byte swizzle) + bulk copy of the packed weight tile
+//               (12288 B) per 128-wide K block into a STAGES-deep ring;
+//   warp 1      TMEM allocator and MMA issuer: 4 MMAs (K = 32 each) per K
+//               block into the int32 partial buffer of the current group
+//               (double buffered, T columns each), commits per group;
+//   warps 2..5  unpack: each thread owns one weight row, turns its 96 packed
+//               bytes into 128 int8 codes (code * 4, the 6-bit field in the
+//               top of each byte) and stores them into a TMEM A slot (4
+//               slots of 32 columns);
+//   warps 6..   epilogue: per group, load the int32 partials from TMEM,
+//               release the buffer, and accumulate
+//               acc += float(P) * (sw[n,g]/4 * sa[m,g]) in FP32 registers;
+//               at the end store FP16 (or reduce across the cluster first).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "flexq_ptx.cuh"
+
+namespace flexq {
+
+constexpr int kTileRows = 128;        // weight rows per tile (MMA M)
+constexpr int kKBlock = 128;          // codes per K block
+constexpr int kWTileBytes = 12288;    // packed bytes of a 128 x 128 tile
+constexpr int kASlots = 4;            // TMEM A ring depth
+constexpr int kStatusTimeout = 5;     // == FLEXQ_ERR_DEVICE_TIMEOUT
+
+struct GemmArgs {
+  const __half* xs;        // [M, G] activation scales
+  const uint8_t* wp;       // packed weights, device form
+  const __half* ws;        // [N, G] weight scales
+  __half* y;               // [M, N] output (GEMM mode)
+  int32_t* p;              // [G, M, N] partials (debug mode)
+  unsigned int* status;    // device status word [4]
+  unsigned long long wait_limit_ns;
+  int M, N, K, gs, split;
+  int ctrl_offset;         // byte offset of the control block in smem
+  int stall;               // test hook: withhold the first stage
+};
+
+template <int T>
+struct GemmCfg {
+  static constexpr int kEpiWarps = (T <= 32) ? 4 : 8;
+  static constexpr int kThreads = (6 + kEpiWarps) * 32;
+  static constexpr int kCols = T / (kEpiWarps / 4);      // tokens per epi warp
+  static constexpr int kStages = (T == 16) ? 7 : (T == 32) ? 6 : (T == 64) ? 5 : 4;
+  static constexpr int kMinBlocks = (T <= 64) ? 2 : 1;
+  static constexpr int kMaxSplit = (T == 16) ? 8 : (T == 32) ? 6 : (T == 64) ? 4 : 2;
+  static constexpr int kXsBytes = T * 128;
+  static constexpr int kStageBytes = kXsBytes + kWTileBytes;
+  static constexpr int kPCol0 = 0;
+  static constexpr int kACol0 = 2 * T;
+  static constexpr int kTmemCols = (2 * T + 128 <= 256) ? 256 : 512;
+  static constexpr int kLdChunk = (T == 128) ? 32 : 16;   // TMEM columns per load batch
+  static_assert(kCols % 16 == 0, "epilogue column chunking");
+};
+
+template <int T>
+struct GemmCtrl {
+  uint64_t full[GemmCfg<T>::kStages];
+  uint64_t empty[GemmCfg<T>::kStages];
+  uint64_t a_full[kASlots];
+  uint64_t a_empty[kASlots];
+  uint64_t p_full[2];
+  uint64_t p_empty[2];
+  uint64_t done;
+  uint32_t tmem_base;
+  uint32_t pad;
+  float sa[GemmCfg<T>::kEpiWarps][GemmCfg<T>::kCols];
+};
+
+__device__ __forceinline__ void record_status(unsigned int* status, int code,
+                                              int where) {
+  if (atomicCAS(status, 0u, static_cast<unsigned>(code)) == 0u) {
+    status[1] = static_cast<unsigned>(where);
+    status[2] = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  }
+}
+
+// All lanes wait; the warp agrees on the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
+                                          uint64_t limit) {
+  const bool ok = mbar_wait(bar, parity, limit);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Four 6-bit codes in the low 24 bits of q (bits above 23 ignored) -> four
+// int8 lanes holding code * 4 (the 6-bit two's-complement field sits in bits
+// [7:2] of each byte).
+__device__ __forceinline__ uint32_t expand_quad(uint32_t q) {
+  const uint32_t t = (q & 0x0000FFFFu) | ((q << 4) & 0xFFFF0000u);
+  return ((t << 2) & 0x00FC00FCu) | ((t << 4) & 0xFC00FC00u);
+}
+
+// 12 canonical packed words (16 quads, 64 codes) -> 16 int8x4 words.
+__device__ __forceinline__ void unpack48(const uint32_t (&w)[12],
+                                         uint32_t (&out)[16]) {
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint32_t w0 = w[3 * t], w1 = w[3 * t + 1], w2 = w[3 * t + 2];
+    out[4 * t + 0] = expand_quad(w0);
+    out[4 * t + 1] = expand_quad(__funnelshift_r(w0, w1, 24));
+    out[4 * t + 2] = expand_quad(__funnelshift_r(w1, w2, 16));
+    out[4 * t + 3] = expand_quad(w2 >> 8);
+  }
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, "
+      "%7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+      "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]),
+      "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+template <int T, bool PARTIALS>
+__global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
+    gemm_w6ax_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
+  using Cfg = GemmCfg<T>;
+  constexpr int STAGES = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* xs_ring = base;                                  // STAGES * kXsBytes
+  uint8_t* w_ring = base + STAGES * Cfg::kXsBytes;          // STAGES * 12288
+  float* red = reinterpret_cast<float*>(base);              // cluster reduction
+  GemmCtrl<T>* ctrl = reinterpret_cast<GemmCtrl<T>*>(base + args.ctrl_offset);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t lim = args.wait_limit_ns;
+
+  const int ks = blockIdx.x;            // K split index == rank in cluster
+  const int nt = blockIdx.y;            // weight tile
+  const int mt = blockIdx.z;            // token tile
+  const int M = args.M, N = args.N, K = args.K, gs = args.gs, S = args.split;
+  const int KB = K / kKBlock;
+  const int U = gs > kKBlock ? gs / kKBlock : 1;      // K blocks per split unit
+  const int units = KB / U;
+  const int u0 = static_cast<int>((static_cast<long long>(ks) * units) / S);
+  const int u1 = static_cast<int>((static_cast<long long>(ks + 1) * units) / S);
+  const int kb0 = u0 * U;
+  const int nkb = (u1 - u0) * U;
+  const int G = K / gs;
+  const int g0 = kb0 * kKBlock / gs;
+  const int ngroups = nkb * kKBlock / gs;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ctrl->full[s], 1);
+      mbar_init(&ctrl->empty[s], 4 + 1);     // 4 unpack warps + MMA commit
+    }
+    for (int s = 0; s < kASlots; ++s) {
+      mbar_init(&ctrl->a_full[s], 4);
+      mbar_init(&ctrl->a_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctrl->p_full[b], 1);
+      mbar_init(&ctrl->p_empty[b], Cfg::kEpiWarps);
+    }
+    mbar_init(&ctrl->done, 1);
+    fence_barrier_init();
+    prefetch_tensormap(&tmap_x);
+  }
+  if (warp == 1) tmem_alloc(&ctrl->tmem_base, Cfg::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+
+  // epilogue state lives across the role switch below
+  float acc[Cfg::kCols];
+#pragma unroll
+  for (int j = 0; j < Cfg::kCols; ++j) acc[j] = 0.0f;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- producer ----
+    if (lane == 0) {
+      uint32_t issued = 0, parity = 0;
+      bool ok = true;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % STAGES;
+        if (i >= STAGES &&
+            !mbar_wait(&ctrl->empty[s], ((i / STAGES) - 1) & 1, lim)) {
+          ok = false;
+          break;
+        }
+        if (args.stall && i == 0) continue;
+        mbar_arrive_expect_tx(&ctrl->full[s], Cfg::kStageBytes);
+        tma_load_2d(xs_ring + s * Cfg::kXsBytes, &tmap_x, &ctrl->full[s],
+                    (kb0 + i) * kKBlock, mt * T);
+        bulk_load(w_ring + s * kWTileBytes,
+                  args.wp + (static_cast<size_t>(nt) * KB + kb0 + i) * kWTileBytes,
+                  kWTileBytes, &ctrl->full[s]);
+        issued |= 1u << s;
+        parity = (parity & ~(1u << s)) | (static_cast<uint32_t>((i / STAGES) & 1) << s);
+      }
+      if (!ok) record_status(args.status, kStatusTimeout, 0);
+      // every issued copy must land before the CTA may finish
+      for (int s = 0; s < STAGES; ++s)
+        if ((issued >> s) & 1u) mbar_wait(&ctrl->full[s], (parity >> s) & 1u, lim);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA -----
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(kTileRows, T);
+      int lg = 0;
+      bool ok = true;
+      for (int i = 0; i < nkb && ok; ++i) {
+        const int s = i % STAGES;
+        const int slot = i & (kASlots - 1);
+        if (!mbar_wait(&ctrl->full[s], (i / STAGES) & 1, lim) ||
+            !mbar_wait(&ctrl->a_full[slot], (i / kASlots) & 1, lim)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t xs_addr = smem_u32(xs_ring + s * Cfg::kXsBytes);
+#pragma unroll
+        for (int sub = 0; sub < 4; ++sub) {
+          const int kk = (kb0 + i) * kKBlock + sub * 32;
+          const bool first = (kk % gs) == 0;
+          const bool last = ((kk + 32) % gs) == 0;
+          const int b = lg & 1;
+          if (first && lg >= 2) {
+            if (!mbar_wait(&ctrl->p_empty[b], ((lg >> 1) - 1) & 1, lim)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          mma_i8_tmem_a(tmem + Cfg::kPCol0 + b * T,
+                        tmem + Cfg::kACol0 + slot * 32 + sub * 8,
+                        smem_desc_k_sw128(xs_addr + sub * 32), idesc,
+                        first ? 0u : 1u);
+          if (last) {
+            mma_commit(&ctrl->p_full[b]);
+            ++lg;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&ctrl->empty[s]);
+        mma_commit(&ctrl->a_empty[slot]);
+      }
+      if (!ok) record_status(args.status, kStatusTimeout, 1);
+      // all issued MMAs must finish before TMEM is released
+      mma_commit(&ctrl->done);
+      mbar_wait(&ctrl->done, 0, lim);
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // -------------------------------------------------------- unpack -----
+    const int q = warp & 3;                       // TMEM lane quarter
+    const int row = q * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % STAGES;
+      if (!warp_wait(&ctrl->full[s], (i / STAGES) & 1, lim)) {
+        if (lane == 0) record_status(args.status, kStatusTimeout, 2);
+        break;
+      }
+      const uint4* src = reinterpret_cast<const uint4*>(w_ring + s * kWTileBytes) + row;
+      uint32_t wa[12], wb[12];
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        const uint4 a = src[j * 128];
+        const uint4 b = src[(j + 3) * 128];
+        wa[4 * j] = a.x; wa[4 * j + 1] = a.y; wa[4 * j + 2] = a.z; wa[4 * j + 3] = a.w;
+        wb[4 * j] = b.x; wb[4 * j + 1] = b.y; wb[4 * j + 2] = b.z; wb[4 * j + 3] = b.w;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctrl->empty[s]);
+      const int slot = i & (kASlots - 1);
+      if (i >= kASlots &&
+          !warp_wait(&ctrl->a_empty[slot], ((i / kASlots) - 1) & 1, lim)) {
+        if (lane == 0) record_status(args.status, kStatusTimeout, 3);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t col = tmem + lane_base + Cfg::kACol0 + slot * 32;
+      uint32_t out[16];
+      unpack48(wa, out);
+      tmem_st16(col, out);
+      unpack48(wb, out);
+      tmem_st16(col + 16, out);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctrl->a_full[slot]);
+    }
+  } else {
+    // ------------------------------------------------------ epilogue -----
+    const int e = warp - 6;
+    const int q = warp & 3;
+    const int c = e >> 2;
+    const int row = q * 32 + lane;
+    const int n = nt * kTileRows + row;
+    const int col0 = c * Cfg::kCols;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    float* sa_w = ctrl->sa[e];
+    const int m_base = mt * T + col0;
+    // activation scales of this warp's tokens for a group: lane l holds
+    // tokens col0 + l and col0 + l + 32
+    auto load_sa = [&](int g, float (&v)[2]) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = lane + 32 * h;
+        const int m = m_base + t;
+        v[h] = (t < Cfg::kCols && m < M)
+                   ? __half2float(args.xs[static_cast<size_t>(m) * G + g])
+                   : 0.0f;
+      }
+    };
+    float sa_next[2] = {0.0f, 0.0f};
+    float sw_next = 0.0f;
+    if (ngroups > 0) {
+      if (!PARTIALS) load_sa(g0, sa_next);
+      if (!PARTIALS) sw_next = __half2float(args.ws[static_cast<size_t>(n) * G + g0]);
+    }
+    for (int lg = 0; lg < ngroups; ++lg) {
+      const int b = lg & 1;
+      const int g = g0 + lg;
+      float swn = 0.0f;
+      if (!PARTIALS) {
+        __syncwarp();
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          if (lane + 32 * h < Cfg::kCols) sa_w[lane + 32 * h] = sa_next[h];
+        __syncwarp();
+        swn = sw_next * 0.25f;               // codes in TMEM are 4 * code
+        if (lg + 1 < ngroups) {
+          load_sa(g + 1, sa_next);
+          sw_next = __half2float(args.ws[static_cast<size_t>(n) * G + g + 1]);
+        }
+      }
+      if (!warp_wait(&ctrl->p_full[b], (lg >> 1) & 1, lim)) {
+        if (lane == 0) record_status(args.status, kStatusTimeout, 4);
+        break;
+      }
+      tc_fence_after();
+      // drain the partials in chunks; the buffer is released right after the
+      // last chunk has been read, before that chunk's arithmetic
+      constexpr int CH = Cfg::kLdChunk;
+#pragma unroll
+      for (int ch = 0; ch < Cfg::kCols / CH; ++ch) {
+        uint32_t pv[CH];
+#pragma unroll
+        for (int h = 0; h < CH / 16; ++h) {
+          uint32_t (&r)[16] = *reinterpret_cast<uint32_t(*)[16]>(&pv[16 * h]);
+          tmem_ld16(tmem + lane_base + Cfg::kPCol0 + b * T + col0 + ch * CH + 16 * h, r);
+        }
+        tmem_wait_ld();
+        if (ch == Cfg::kCols / CH - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctrl->p_empty[b]);
+        }
+        if (PARTIALS) {
+#pragma unroll
+          for (int j = 0; j < CH; ++j) {
+            const int m = m_base + ch * CH + j;
+            if (m < M)
+              args.p[(static_cast<size_t>(g) * M + m) * N + n] =
+                  static_cast<int32_t>(pv[j]) >> 2;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < CH; ++j)
+            acc[ch * CH + j] = fmaf(static_cast<float>(static_cast<int32_t>(pv[j])),
+                                    swn * sa_w[ch * CH + j], acc[ch * CH + j]);
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown --
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+  if (PARTIALS) return;
+
+  const bool is_epi = warp >= 6;
+  const int e = warp - 6;
+  const int row = (warp & 3) * 32 + lane;
+  const int col0 = (e >> 2) * Cfg::kCols;
+  if (S > 1) {
+    // split-K: ranks 1..S-1 add their partial tiles into rank 0's shared
+    // memory (the stage ring is idle now), in a fixed order
+    cluster_sync_all();
+    if (is_epi && ks != 0) {
+      const uint32_t remote = map_to_rank(smem_u32(red), 0);
+#pragma unroll
+      for (int j = 0; j < Cfg::kCols; ++j) {
+        const uint32_t off = static_cast<uint32_t>(((ks - 1) * T + col0 + j) * kTileRows + row);
+        st_cluster_f32(remote + off * 4u, acc[j]);
+      }
+    }
+    cluster_sync_all();
+    if (ks != 0) return;
+    if (is_epi) {
+      for (int r = 1; r < S; ++r) {
+#pragma unroll
+        for (int j = 0; j < Cfg::kCols; ++j)
+          acc[j] += red[((r - 1) * T + col0 + j) * kTileRows + row];
+      }
+    }
+  }
+  if (is_epi) {
+    const int n = nt * kTileRows + row;
+#pragma unroll
+    for (int j = 0; j < Cfg::kCols; ++j) {
+      const int m = mt * T + col0 + j;
+      if (m < M) args.y[static_cast<size_t>(m) * N + n] = __float2half_rn(acc[j]);
+    }
+  }
+}
+
+}  // namespace flexq

@@ -1,0 +1,196 @@
+"""Python binding of libflexq.so (the C ABI in include/flexq.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  torch supplies device memory and the current CUDA stream.  There is
+no fallback: if the library is missing or a call fails, an exception is
+raised.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libflexq.so")
+
+FLEXQ_OK = 0
+FLEXQ_ERR_INVALID_ARG = 1
+FLEXQ_ERR_UNSUPPORTED = 2
+FLEXQ_ERR_MISALIGNED = 3
+FLEXQ_ERR_CUDA = 4
+FLEXQ_ERR_DEVICE_TIMEOUT = 5
+
+_lib = None
+
+
+class FlexQError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(message)
+        self.status = status
+
+
+def lib():
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m bit_group_quantized_flexq_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        c_int, c_void_p, c_size_t = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+        sig = {
+            "flexq_status_string": (ctypes.c_char_p, [c_int]),
+            "flexq_last_error_message": (ctypes.c_char_p, []),
+            "flexq_weight_packed_bytes": (c_size_t, [c_int, c_int, c_int]),
+            "flexq_quantize_weight": (c_int, [c_int, c_int, c_int, c_void_p, c_void_p,
+                                              c_void_p, c_void_p]),
+            "flexq_quantize_act": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p,
+                                           c_void_p, c_void_p]),
+            "flexq_gemm_w6a6": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p,
+                                        c_void_p, c_void_p, c_void_p, c_void_p]),
+            "flexq_gemm_w6a8": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p,
+                                        c_void_p, c_void_p, c_void_p, c_void_p]),
+            "flexq_debug_group_partials": (c_int, [c_int, c_int, c_int, c_int, c_void_p,
+                                                   c_void_p, c_void_p, c_void_p]),
+            "flexq_gemm_plan": (c_int, [c_int, c_int, c_int, c_int,
+                                        ctypes.POINTER(c_int), ctypes.POINTER(c_int),
+                                        ctypes.POINTER(c_int)]),
+            "flexq_debug_force_plan": (c_int, [c_int, c_int]),
+            "flexq_set_wait_limit_ns": (c_int, [ctypes.c_uint64]),
+            "flexq_debug_inject_stall": (c_int, [c_int]),
+            "flexq_get_device_status": (c_int, [c_void_p]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status):
+    if status != FLEXQ_OK:
+        L = lib()
+        name = L.flexq_status_string(status).decode()
+        detail = L.flexq_last_error_message().decode()
+        raise FlexQError(status, f"{name}: {detail}")
+
+
+def _stream(t=None):
+    dev = t.device if t is not None else torch.device("cuda")
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, name, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must live on a CUDA device")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def weight_packed_bytes(N, K, group_size):
+    return int(lib().flexq_weight_packed_bytes(N, K, group_size))
+
+
+def quantize_weight(w, group_size, out=None):
+    """FP16 W [N, K] -> (packed uint8 [3NK/4] in the device form, FP16 scales [N, K/gs])."""
+    _need(w, "w", torch.float16)
+    N, K = w.shape
+    nbytes = weight_packed_bytes(N, K, group_size)
+    if nbytes == 0:
+        raise FlexQError(FLEXQ_ERR_UNSUPPORTED, f"unsupported weight shape {N}x{K}, gs={group_size}")
+    if out is None:
+        out = (torch.empty(nbytes, dtype=torch.uint8, device=w.device),
+               torch.empty(N, K // group_size, dtype=torch.float16, device=w.device))
+    wp, ws = out
+    _need(wp, "packed", torch.uint8, (nbytes,))
+    _need(ws, "scales", torch.float16, (N, K // group_size))
+    _check(lib().flexq_quantize_weight(N, K, group_size, _ptr(w), _ptr(wp), _ptr(ws), _stream(w)))
+    return wp, ws
+
+
+def quantize_act(x, group_size, bits, out=None):
+    """FP16 X [M, K] -> (int8 codes [M, K], FP16 scales [M, K/gs])."""
+    _need(x, "x", torch.float16)
+    M, K = x.shape
+    if out is None:
+        out = (torch.empty(M, K, dtype=torch.int8, device=x.device),
+               torch.empty(M, K // group_size, dtype=torch.float16, device=x.device))
+    xq, xs = out
+    _need(xq, "codes", torch.int8, (M, K))
+    _need(xs, "scales", torch.float16, (M, K // group_size))
+    _check(lib().flexq_quantize_act(M, K, group_size, bits, _ptr(x), _ptr(xq), _ptr(xs), _stream(x)))
+    return xq, xs
+
+
+def gemm(xq, xs, wp, ws, N, group_size, act_bits=6, out=None):
+    """Y [M, N] FP16 = dequant(xq, xs) . dequant(wp, ws)^T (W6A6 or W6A8)."""
+    _need(xq, "xq", torch.int8)
+    M, K = xq.shape
+    _need(xs, "xs", torch.float16, (M, K // group_size))
+    _need(wp, "wp", torch.uint8, (weight_packed_bytes(N, K, group_size),))
+    _need(ws, "ws", torch.float16, (N, K // group_size))
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.float16, device=xq.device)
+    _need(out, "out", torch.float16, (M, N))
+    fn = {6: lib().flexq_gemm_w6a6, 8: lib().flexq_gemm_w6a8}[act_bits]
+    _check(fn(M, N, K, group_size, _ptr(xq), _ptr(xs), _ptr(wp), _ptr(ws), _ptr(out), _stream(xq)))
+    return out
+
+
+def debug_group_partials(xq, wp, N, group_size, out=None):
+    """int32 [G, M, N] per-group integer partials from the GEMM mainloop."""
+    _need(xq, "xq", torch.int8)
+    M, K = xq.shape
+    G = K // group_size
+    if out is None:
+        out = torch.empty(G, M, N, dtype=torch.int32, device=xq.device)
+    _need(out, "out", torch.int32, (G, M, N))
+    _check(lib().flexq_debug_group_partials(M, N, K, group_size, _ptr(xq), _ptr(wp), _ptr(out),
+                                            _stream(xq)))
+    return out
+
+
+def linear(x, wp, ws, N, group_size, act_bits=6, xq_out=None, y_out=None):
+    """One linear layer on FP16 activations: quantize X, then the group GEMM."""
+    xq, xs = quantize_act(x, group_size, act_bits, out=xq_out)
+    return gemm(xq, xs, wp, ws, N, group_size, act_bits, out=y_out)
+
+
+def plan(M, N, K, group_size):
+    """(tokens per tile, K split, CTAs) of the GEMM launch for a shape."""
+    t, s, c = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(lib().flexq_gemm_plan(M, N, K, group_size, ctypes.byref(t), ctypes.byref(s),
+                                 ctypes.byref(c)))
+    return t.value, s.value, c.value
+
+
+def force_plan(tile_tokens=0, k_split=0):
+    _check(lib().flexq_debug_force_plan(tile_tokens, k_split))
+
+
+def set_wait_limit_ns(ns):
+    _check(lib().flexq_set_wait_limit_ns(int(ns)))
+
+
+def inject_stall(enable=True):
+    _check(lib().flexq_debug_inject_stall(1 if enable else 0))
+
+
+def device_status(device=None):
+    """Synchronizes the current stream and returns (status, message); clears it."""
+    s = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    st = lib().flexq_get_device_status(s)
+    return st, lib().flexq_last_error_message().decode()

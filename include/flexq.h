@@ -1,0 +1,180 @@
+/*
+ * flexq.h -- C ABI of the B200 (sm_100a) library for FlexQ's group-quantized
+ * W6A6 / W6A8 linear layer.
+ *
+ * The method (FlexQ: Efficient Post-training INT6 Quantization for LLM
+ * Serving via Algorithm-System Co-Design): weights are quantized uniformly to
+ * 6 bits, activations to 6 bits or, in sensitive layers, 8 bits (arXiv
+ * abstract); both use fine-grained groups along K that share one scale
+ * (drgamma blog, "Fine-Grained Quantization and Layer Sensitivity" and
+ * "Bridging Software and Hardware with BTC"); the GEMM sums integer products
+ * per group and recombines them with the scales, with dequantization fused
+ * into the GEMM (blog, "Bridging Software and Hardware with BTC").
+ *
+ * Conventions shared by every entry point
+ *   - All buffers are DEVICE memory owned by the caller; the library never
+ *     allocates, frees or retains them.  FP16 buffers are IEEE binary16.
+ *   - Matrices are row-major.  M = tokens, N = output channels, K = input
+ *     channels, gs = group size along K, G = K / gs.
+ *   - Supported shapes: M >= 0 (M == 0 is a no-op), N % 128 == 0, K % 128 == 0,
+ *     gs in {32, 64, 128, 256}, K % gs == 0.
+ *   - Every device pointer must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     are asynchronous: they validate their arguments, enqueue the work on
+ *     `stream` and return.  Invalid arguments are reported before anything
+ *     is enqueued.
+ *   - Return value: a flexq_status_t.  flexq_last_error_message() gives a
+ *     human-readable detail for the calling thread's last failure.
+ *   - Device-side failures (a pipeline wait that exceeded its time limit) do
+ *     not trap: the kernel records them in a device status word and returns;
+ *     flexq_get_device_status() reads and clears that word.
+ */
+#ifndef FLEXQ_H_
+#define FLEXQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FLEXQ_OK = 0,
+  FLEXQ_ERR_INVALID_ARG = 1,     /* null pointer, negative size, bad bits     */
+  FLEXQ_ERR_UNSUPPORTED = 2,     /* shape outside the supported set above     */
+  FLEXQ_ERR_MISALIGNED = 3,      /* a device pointer is not 16-byte aligned   */
+  FLEXQ_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed      */
+  FLEXQ_ERR_DEVICE_TIMEOUT = 5   /* a kernel's bounded wait gave up           */
+} flexq_status_t;
+
+/* Name of a status code (static string, never NULL). */
+const char* flexq_status_string(int status);
+
+/* Detail of the calling thread's most recent failure ("" if none). */
+const char* flexq_last_error_message(void);
+
+/*
+ * Size in bytes of the packed 6-bit weight buffer for an [N, K] layer:
+ * 3*N*K/4 (four codes in three bytes).  Returns 0 for unsupported shapes.
+ */
+size_t flexq_weight_packed_bytes(int N, int K, int group_size);
+
+/*
+ * flexq_quantize_weight -- offline 6-bit weight quantization and packing.
+ * Passage: uniform 6-bit weights (arXiv abstract); groups along K sharing a
+ * scale (blog, "Fine-Grained Quantization and Layer Sensitivity";
+ * "Bridging Software and Hardware with BTC").
+ *
+ *   W_fp16        [N, K] FP16, finite values.
+ *   Wq_packed     out, flexq_weight_packed_bytes(N, K, gs) bytes: the device
+ *                 form of the 6-bit codes.  Canonical packing: codes c0..c3 at
+ *                 k = 4j..4j+3 of a row give the 24-bit little-endian word
+ *                 (c0&63) | (c1&63)<<6 | (c2&63)<<12 | (c3&63)<<18.  Device
+ *                 form: tiles of 128 rows x 128 codes (12288 bytes), tile
+ *                 (nt, kb) at byte offset (nt*(K/128) + kb)*12288; inside a
+ *                 tile, byte b of 16-byte chunk j (0..5) of row r holds
+ *                 canonical byte kb*96 + 16*j + b of row nt*128 + r and sits
+ *                 at offset (j*128 + r)*16 + b.
+ *   W_scales_fp16 out, [N, G] FP16: s = fp16_rne(absmax / 31) per (n, group),
+ *                 absmax/31 computed as an IEEE FP32 division.
+ * Codes: clamp(round_half_even(w / s), -31, 31) with an IEEE FP32 division by
+ * the stored FP16 scale; a group whose FP16 scale is 0 gets all-zero codes.
+ */
+int flexq_quantize_weight(int N, int K, int group_size, const void* W_fp16,
+                          void* Wq_packed, void* W_scales_fp16, void* stream);
+
+/*
+ * flexq_quantize_act -- per-forward activation quantization, 6 or 8 bits.
+ * Passage: 6-bit activations, 8-bit ones kept in sensitive layers (arXiv
+ * abstract; blog, "Fine-Grained Quantization and Layer Sensitivity").
+ *
+ *   X_fp16        [M, K] FP16, finite values.
+ *   bits          6 (codes in [-31, 31], Q = 31) or 8 (codes in [-127, 127],
+ *                 Q = 127).
+ *   Xq            out, [M, K] int8, one code per byte for both widths.
+ *   X_scales_fp16 out, [M, G] FP16: fp16_rne(absmax / Q) per (m, group).
+ * Same rounding rules as flexq_quantize_weight.
+ */
+int flexq_quantize_act(int M, int K, int group_size, int bits,
+                       const void* X_fp16, int8_t* Xq, void* X_scales_fp16,
+                       void* stream);
+
+/*
+ * flexq_gemm_w6a6 / flexq_gemm_w6a8 -- Y = dequant(Xq) . dequant(Wq)^T.
+ * Passage: the W6A6 / W6A8 GEMM whose integer products are summed per group
+ * and recombined with the scales, dequantization fused into the GEMM (arXiv
+ * abstract; blog, "Bridging Software and Hardware with BTC").
+ *
+ *   Xq, X_scales     activation codes [M, K] int8 and FP16 scales [M, G].
+ *   Wq_packed,       weight codes in the device form above and FP16 scales
+ *   W_scales         [N, G], as written by flexq_quantize_weight.
+ *   Y_fp16           out, [M, N] FP16.
+ * For each group g the integer partial P_g[m,n] = sum_{k in g} Xq[m,k]*Wq[n,k]
+ * is formed exactly (int32), then Y[m,n] = fp16_rne(sum_g P_g[m,n] *
+ * sa[m,g] * sw[n,g]) with the sum over groups accumulated in FP32 (per
+ * output, |Y - Y_exact| <= 5e-4 * max|Y| on the benchmark distributions).
+ * The two entry points run the same kernel: they differ only in the code
+ * range the caller's activations are expected to use ([-31, 31] vs
+ * [-127, 127]); neither checks the range, and any int8 activation code and
+ * any 6-bit weight code (including -32) are multiplied exactly.
+ */
+int flexq_gemm_w6a6(int M, int N, int K, int group_size, const int8_t* Xq,
+                    const void* X_scales, const void* Wq_packed,
+                    const void* W_scales, void* Y_fp16, void* stream);
+int flexq_gemm_w6a8(int M, int N, int K, int group_size, const int8_t* Xq,
+                    const void* X_scales, const void* Wq_packed,
+                    const void* W_scales, void* Y_fp16, void* stream);
+
+/*
+ * flexq_debug_group_partials -- exports the per-group int32 partials of the
+ * GEMM above, computed by the same kernel mainloop (test hook).
+ *   P  out, int32 [G, M, N]: P[g][m][n] = sum_{k in g} Xq[m,k] * Wq[n,k].
+ */
+int flexq_debug_group_partials(int M, int N, int K, int group_size,
+                               const int8_t* Xq, const void* Wq_packed,
+                               int32_t* P, void* stream);
+
+/*
+ * flexq_gemm_plan -- the launch the GEMM entry points would use for a shape:
+ * tokens per tile (16, 32, 64 or 128), K-split factor (CTAs of one cluster
+ * that share an output tile) and the number of CTAs.  Any output pointer may
+ * be NULL.  Pure host computation.
+ */
+int flexq_gemm_plan(int M, int N, int K, int group_size, int* tile_tokens,
+                    int* k_split, int* ctas);
+
+/*
+ * flexq_debug_force_plan -- test hook: make subsequent GEMM launches on the
+ * calling process use tile_tokens (16/32/64/128) and k_split (1..8) when the
+ * shape allows it.  (0, 0) restores the automatic choice.
+ */
+int flexq_debug_force_plan(int tile_tokens, int k_split);
+
+/*
+ * flexq_set_wait_limit_ns -- time limit of every bounded pipeline wait in the
+ * GEMM kernel (default 2e9 ns).  A wait that exceeds it records
+ * FLEXQ_ERR_DEVICE_TIMEOUT in the device status word and the kernel returns.
+ */
+int flexq_set_wait_limit_ns(uint64_t limit_ns);
+
+/*
+ * flexq_debug_inject_stall -- test hook: when enabled, the next GEMM launch's
+ * producer warp withholds its first stage, so every consumer's bounded wait
+ * runs out.  The kernel must then report FLEXQ_ERR_DEVICE_TIMEOUT through
+ * flexq_get_device_status() and leave the context usable.  One-shot.
+ */
+int flexq_debug_inject_stall(int enable);
+
+/*
+ * flexq_get_device_status -- synchronizes `stream`, reads the current
+ * device's status word, clears it and returns FLEXQ_OK or the recorded error
+ * (FLEXQ_ERR_DEVICE_TIMEOUT).  A failing CUDA call returns FLEXQ_ERR_CUDA.
+ */
+int flexq_get_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLEXQ_H_ */

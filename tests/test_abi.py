@@ -1,0 +1,100 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that
+include/flexq.h declares, and rejects invalid arguments before touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_group_quantized_flexq_b200 import build as flexq_build
+from bit_group_quantized_flexq_b200 import flexq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    flexq_build.build()
+    return flexq.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "flexq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(flexq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ["flexq_quantize_weight", "flexq_quantize_act", "flexq_gemm_w6a6",
+                     "flexq_gemm_w6a8", "flexq_debug_group_partials",
+                     "flexq_get_device_status", "flexq_weight_packed_bytes"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    assert L.flexq_status_string(0) == b"FLEXQ_OK"
+    assert L.flexq_status_string(5) == b"FLEXQ_ERR_DEVICE_TIMEOUT"
+    assert L.flexq_status_string(99) == b"FLEXQ_ERR_UNKNOWN"
+
+
+def test_packed_size(L):
+    assert L.flexq_weight_packed_bytes(4096, 4096, 128) == 4096 * 4096 * 3 // 4
+    assert L.flexq_weight_packed_bytes(28672, 8192, 32) == 28672 * 8192 * 3 // 4
+    assert L.flexq_weight_packed_bytes(100, 4096, 128) == 0        # N % 128
+    assert L.flexq_weight_packed_bytes(128, 4096, 48) == 0         # bad gs
+    assert L.flexq_weight_packed_bytes(128, 192, 64) == 0          # K % 128
+
+
+FAKE = ctypes.c_void_p(1 << 20)          # never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p((1 << 20) + 8)
+NULL = ctypes.c_void_p(0)
+
+
+def test_validation_before_any_launch(L):
+    # bad bit width
+    assert L.flexq_quantize_act(4, 256, 128, 7, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert b"bits" in L.flexq_last_error_message()
+    # bad group size / K not a multiple of the group
+    assert L.flexq_quantize_act(4, 256, 48, 6, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
+    assert L.flexq_quantize_act(4, 160, 64, 6, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
+    # null and misaligned pointers
+    assert L.flexq_quantize_act(4, 256, 128, 6, NULL, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert L.flexq_quantize_act(4, 256, 128, 6, FAKE, MISALIGNED, FAKE, NULL) == flexq.FLEXQ_ERR_MISALIGNED
+    # negative sizes
+    assert L.flexq_quantize_act(-1, 256, 128, 6, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    # GEMM shape rules
+    g = L.flexq_gemm_w6a6
+    assert g(4, 200, 256, 128, FAKE, FAKE, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
+    assert g(4, 256, 200, 128, FAKE, FAKE, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
+    assert g(4, 256, 384, 256, FAKE, FAKE, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
+    assert g(4, 256, 256, 128, FAKE, NULL, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert g(4, 256, 256, 128, FAKE, FAKE, FAKE, FAKE, MISALIGNED, NULL) == flexq.FLEXQ_ERR_MISALIGNED
+    assert L.flexq_gemm_w6a8(-3, 256, 256, 128, FAKE, FAKE, FAKE, FAKE, FAKE, NULL) == \
+        flexq.FLEXQ_ERR_INVALID_ARG
+    w = L.flexq_quantize_weight
+    assert w(130, 256, 128, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
+    assert w(128, 256, 128, FAKE, NULL, FAKE, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert L.flexq_debug_force_plan(48, 0) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert L.flexq_debug_force_plan(16, 9) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert L.flexq_set_wait_limit_ns(0) == flexq.FLEXQ_ERR_INVALID_ARG
+
+
+def test_plan_is_host_only_and_sane(L):
+    # tokens per tile follow M; K splits fill the machine at decode sizes
+    for M, T in [(1, 16), (16, 16), (17, 32), (64, 64), (65, 128), (2048, 128)]:
+        t, s, c = flexq.plan(M, 4096, 4096, 128)
+        assert t == T
+        assert 1 <= s <= 8
+        assert c == s * (4096 // 128) * ((M + t - 1) // t)
+    t, s, c = flexq.plan(1, 4096, 4096, 128)
+    assert s > 1                      # 32 weight tiles alone would idle most SMs
+    t, s, c = flexq.plan(1, 4096, 256, 256)
+    assert s == 1                     # one group: nothing to split
+    assert flexq.plan(0, 256, 256, 128) == (0, 0, 0)
