@@ -1,0 +1,590 @@
+#!/usr/bin/env python
+"""Benchmark of the W6A6 group-quantized linear layers of a LLaMA-2-7B block.
+
+Workload (one "step"): for every M in {1, 16, 256, 2048} and every linear layer
+of a LLaMA-2-7B transformer block (q, k, v, o: 4096x4096; gate, up: 11008x4096;
+down: 4096x11008), quantize the FP16 activations to 6-bit group codes (group
+size 128) and run the W6A6 group GEMM against 6-bit packed weights.  Inputs are
+seeded synthetic tensors of those shapes (weights N(0, 0.02); activations
+N(0, 1) with 1% outlier channels x20); every step streams 151 MB of distinct
+packed weights, more than the 126 MB L2, so each GEMM reads its weights from
+HBM.
+
+Output: one JSON line (rank 0).  `value` is whole-job TOPS (2*M*N*K summed over
+the step, divided by the device time), measured over CUDA-graph replays of the
+step with inputs resident in HBM; `e2e` is the same metric through the public
+Python API with host buffers (pinned H2D copy of every layer input, D2H copy of
+every output) inside the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl flexq|reference]
+
+`--impl reference` times the CPU oracle (the plain restatement of the method
+used by the tests) on a bounded sample of the same workload.  With --gpus N > 1
+(launched by torchrun) every rank runs its own replica of the workload (weak
+scaling, no collective on the data path); ranks meet only for the barrier and
+the max-over-ranks timing.
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("W6A6/W6A8 linear-layer TOPS and % of roofline "
+          "(HBM at small M, INT8 peak at large M)")
+UNIT = "TOPS"
+GS = 128
+ACT_BITS = 6
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 2.0          # nominal dense ratio (4.5 vs 2.25 PFLOP/s)
+
+
+# ------------------------------------------------------------- workload ----
+def workload_shapes(ms=None, layers=None):
+    from bit_group_quantized_flexq_b200 import inputs
+    ms = list(ms) if ms else list(inputs.LLAMA2_7B_M)
+    lay = [l for l in inputs.LLAMA2_7B_LAYERS if not layers or l[0] in layers]
+    return ms, lay
+
+
+def step_ops(ms, layers):
+    return sum(2.0 * M * N * K for M in ms for (_, N, K) in layers)
+
+
+def gemm_bytes(M, N, K, gs=GS):
+    """Algorithmic HBM bytes of one GEMM launch: packed weights (0.75 B per
+    element), weight scales, int8 activation codes and scales, FP16 output."""
+    return 0.75 * N * K + 2.0 * N * K / gs + M * K + 2.0 * M * K / gs + 2.0 * M * N
+
+
+def workload_name(ms, layers):
+    return ("LLaMA-2-7B block W6A6 linear layers ("
+            + ",".join(f"{n}:{N}x{K}" for n, N, K in layers)
+            + f"), group 128, M in {{{','.join(map(str, ms))}}}")
+
+
+# ------------------------------------------------------------ distributed --
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def dist_init(backend):
+    import datetime
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def max_over_ranks(x, device=None):
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate(units_per_rank, world, t_max_s):
+    """Whole-job throughput: the units all ranks processed over the max time."""
+    return units_per_rank * world / t_max_s
+
+
+# ----------------------------------------------------------------- clocks --
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        return self.summary()
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_digest():
+    h = hashlib.sha256()
+    for f in ("flexq_gemm.cuh", "flexq_ptx.cuh", "flexq_api.cu"):
+        with open(os.path.join(ROOT, "bit_group_quantized_flexq_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the dominant GEMM from the committed ncu
+    summary, or None when the kernel source changed since that capture."""
+    p = os.path.join(ROOT, "profiles", "gemm_m2048_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("kernel_src_sha") != kernel_source_digest():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------ flexq arm ----
+class Layers:
+    """Device-resident workload: packed weights, activations, outputs."""
+
+    def __init__(self, ms, layers, device):
+        import torch
+        from bit_group_quantized_flexq_b200 import flexq, inputs
+        self.ms, self.layers, self.dev = ms, layers, device
+        self.w = []
+        for name, N, K in layers:
+            w16 = inputs.weights(N, K, std=0.02, seed=inputs.layer_seed("7b", name)).to(device)
+            wp, ws = flexq.quantize_weight(w16, GS)
+            del w16
+            self.w.append((name, N, K, wp, ws))
+        self.x, self.xq, self.xs, self.y = {}, {}, {}, {}
+        for M in ms:
+            for K in sorted({K for (_, _, K) in layers}):
+                x = inputs.activations(M, K, outlier_frac=0.01, outlier_scale=20.0,
+                                       seed=inputs.layer_seed("7b-x", M, K))
+                self.x[(M, K)] = x.to(device)
+                self.xq[(M, K)] = torch.empty(M, K, dtype=torch.int8, device=device)
+                self.xs[(M, K)] = torch.empty(M, K // GS, dtype=torch.float16, device=device)
+            for (name, N, K) in layers:
+                self.y[(M, name)] = torch.empty(M, N, dtype=torch.float16, device=device)
+        torch.cuda.synchronize(device)
+
+    def launches_per_step(self):
+        return 2 * len(self.ms) * len(self.w)
+
+    def step(self, marks=None, gemm_marks=None, dominant_m=None):
+        """One pass of the hot path.  marks: events recorded at the start and
+        after each M group; gemm_marks: (start, end) events around each GEMM
+        of the dominant M."""
+        from bit_group_quantized_flexq_b200 import flexq
+        gi = 0
+        if marks is not None:
+            marks[0].record()
+        for mi, M in enumerate(self.ms):
+            for (name, N, K, wp, ws) in self.w:
+                xq, xs = flexq.quantize_act(self.x[(M, K)], GS, ACT_BITS,
+                                            out=(self.xq[(M, K)], self.xs[(M, K)]))
+                timed = gemm_marks is not None and M == dominant_m
+                if timed:
+                    gemm_marks[gi][0].record()
+                flexq.gemm(xq, xs, wp, ws, N, GS, ACT_BITS, out=self.y[(M, name)])
+                if timed:
+                    gemm_marks[gi][1].record()
+                    gi += 1
+            if marks is not None:
+                marks[mi + 1].record()
+
+
+def run_flexq(args, rank, world):
+    import torch
+    from bit_group_quantized_flexq_b200 import flexq
+    _, _, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    flexq.lib()                                   # fail loudly if not built
+    ms, layers = workload_shapes(args.ms, args.layers)
+    dominant_m = max(ms)
+    W = Layers(ms, layers, device)
+    ops = step_ops(ms, layers)
+    nlay = len(layers)
+
+    def new_events(n):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    # eager warm-up (first calls set kernel attributes; nothing is captured yet)
+    for _ in range(2):
+        W.step()
+    torch.cuda.synchronize(device)
+
+    stream = torch.cuda.Stream(device)
+    graphs, marks, gmarks = [], [], []
+    if args.graph:
+        for i in range(args.steps):
+            mk = new_events(len(ms) + 1)
+            gm = [new_events(2) for _ in range(nlay)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    W.step(mk, gm, dominant_m)
+            graphs.append(g)
+            marks.append(mk)
+            gmarks.append(gm)
+        torch.cuda.synchronize(device)
+
+    def run_step(i):
+        if args.graph:
+            graphs[i].replay()
+        else:
+            W.step(marks[i], gmarks[i], dominant_m)
+
+    if not args.graph:
+        marks = [new_events(len(ms) + 1) for _ in range(args.steps)]
+        gmarks = [[new_events(2) for _ in range(nlay)] for _ in range(args.steps)]
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            run_step(i % max(1, args.steps))
+        torch.cuda.synchronize(device)
+        barrier(device)
+        torch.cuda.synchronize(device)
+        clocks = ClockSampler(device.index if device.index is not None else 0)
+        clocks.start()
+        time.sleep(0.3)                           # sampler up before timing
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            run_step(i)
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+        clock_summary = clocks.stop()
+    barrier(device)
+    elapsed_ms = t0.elapsed_time(t1)
+    t_max_s = max_over_ranks(elapsed_ms / 1e3, device)
+    status, msg = flexq.device_status(device)
+    if status != flexq.FLEXQ_OK:
+        raise RuntimeError(f"device status after the timed region: {msg}")
+
+    # per-M time and dominant-kernel launches, from the events of the timed steps
+    per_m_ms = [statistics.mean(marks[i][mi].elapsed_time(marks[i][mi + 1])
+                                for i in range(args.steps)) for mi in range(len(ms))]
+    dom_durs = [gmarks[i][j][0].elapsed_time(gmarks[i][j][1])
+                for i in range(args.steps) for j in range(nlay)]
+    dom_flops_per_step = sum(2.0 * dominant_m * N * K for (_, N, K) in layers)
+    dom_avg_ms = statistics.mean(dom_durs)
+    dom_flops_per_launch = dom_flops_per_step / nlay
+    achieved_tops = dom_flops_per_launch / (dom_avg_ms / 1e3) / 1e12
+
+    peaks, peak_src = measured_peaks()
+    long_region = elapsed_ms > 1000.0
+    bf16 = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops",
+                     peaks.get("bf16_tflops"))
+    int8_peak = bf16 * INT8_OVER_BF16
+    hbm = peaks["hbm_gbs"]
+
+    per_m = []
+    for mi, M in enumerate(ms):
+        m_ops = sum(2.0 * M * N * K for (_, N, K) in layers)
+        per_m.append({"M": M, "ms": round(per_m_ms[mi], 5),
+                      "tops": round(m_ops / (per_m_ms[mi] / 1e3) / 1e12, 3)})
+
+    # GEMM-only diagnostics per M (after the timed region, not part of value)
+    diag = gemm_diagnostics(W, device, hbm, int8_peak) if args.diag else None
+
+    traffic = profiled_traffic()
+    result = {
+        "metric": METRIC,
+        "value": round(aggregate(ops, world, t_max_s) / 1e12, 3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(t_max_s * 1e3 / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic",
+        "config": {
+            "workload": workload_name(ms, layers),
+            "group_size": GS, "act_bits": ACT_BITS, "weight_bits": 6,
+            "shapes": [[n, N, K] for n, N, K in layers], "M": ms,
+            "ops_per_step": ops,
+            "l2": "inputs larger than L2: each step streams 151 MB of distinct packed weights",
+            "timing": "CUDA-graph replay of each step" if args.graph else "eager launches",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "per_m": per_m,
+        "roofline": {
+            "bound": "tensor",
+            "kernel": f"gemm_w6ax_kernel (M={dominant_m} launches)",
+            "achieved": round(achieved_tops, 2),
+            "peak": round(int8_peak, 1),
+            "unit": "TFLOP/s",
+            "frac": round(achieved_tops / int8_peak, 4),
+            "peak_source": (f"{peak_src}: {'sustained' if long_region else 'burst'} bf16 x "
+                            f"{INT8_OVER_BF16:g} (nominal int8/bf16 dense ratio)"),
+            "avg_launch_us": round(dom_avg_ms * 1e3, 2),
+            "traffic": traffic,
+        },
+        "gpu_launches": W.launches_per_step() * args.steps,
+        "clocks": clock_summary,
+    }
+    if diag:
+        result["gemm_by_m"] = diag
+    if args.e2e:
+        result["e2e"] = run_e2e(W, args, device, world)
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        result["cpu_baseline"] = run_cpu_baseline(args.cpu_budget_s)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    graphs.clear()
+
+
+def gemm_diagnostics(W, device, hbm_gbs, int8_peak_tops, reps=10):
+    """Per-M GEMM-only times and roofline fractions (HBM bound for M <= 16,
+    tensor bound above).  Each GEMM runs `reps` times back to back; the
+    weights of the other layers stream in between, so reads stay cold."""
+    import torch
+    from bit_group_quantized_flexq_b200 import flexq
+    out = []
+    for M in W.ms:
+        durs = {name: [] for (name, _, _, _, _) in W.w}
+        for _ in range(reps):
+            for (name, N, K, wp, ws) in W.w:
+                xq, xs = W.xq[(M, K)], W.xs[(M, K)]
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                flexq.gemm(xq, xs, wp, ws, N, GS, ACT_BITS, out=W.y[(M, name)])
+                e1.record()
+                durs[name].append((e0, e1))
+        torch.cuda.synchronize(device)
+        t_us, bytes_, flops = 0.0, 0.0, 0.0
+        for (name, N, K, _, _) in W.w:
+            d = statistics.median(a.elapsed_time(b) for a, b in durs[name]) * 1e3
+            t_us += d
+            bytes_ += gemm_bytes(M, N, K)
+            flops += 2.0 * M * N * K
+        gbs = bytes_ / (t_us * 1e-6) / 1e9
+        tops = flops / (t_us * 1e-6) / 1e12
+        bound = "hbm" if M <= 16 else "tensor"
+        frac = gbs / hbm_gbs if bound == "hbm" else tops / int8_peak_tops
+        out.append({"M": M, "gemm_us": round(t_us, 2), "GB/s": round(gbs, 1),
+                    "TOPS": round(tops, 2), "bound": bound, "frac": round(frac, 4),
+                    "plan": [list(flexq.plan(M, N, K, GS)) for (_, N, K, _, _) in W.w]})
+    return out
+
+
+def run_e2e(W, args, device, world):
+    """The same metric through the public API with host buffers: every step
+    copies each layer's FP16 input from pinned host memory and each output
+    back to pinned host memory."""
+    import torch
+    from bit_group_quantized_flexq_b200 import flexq
+    hx = {k: v.cpu().pin_memory() for k, v in W.x.items()}
+    hy = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in W.y.items()}
+    dx = {k: torch.empty_like(v) for k, v in W.x.items()}
+    h2d = sum(W.x[(M, K)].numel() * 2 for M in W.ms for (_, _, K, _, _) in W.w)
+    d2h = sum(v.numel() * 2 for v in W.y.values())
+
+    def step():
+        for M in W.ms:
+            for (name, N, K, wp, ws) in W.w:
+                dx[(M, K)].copy_(hx[(M, K)], non_blocking=True)
+                flexq.linear(dx[(M, K)], wp, ws, N, GS, ACT_BITS,
+                             xq_out=(W.xq[(M, K)], W.xs[(M, K)]), y_out=W.y[(M, name)])
+                hy[(M, name)].copy_(W.y[(M, name)], non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize(device)
+    t_max = max_over_ranks(t0.elapsed_time(t1) / 1e3, device)
+    ops = step_ops(W.ms, [(n, N, K) for (n, N, K, _, _) in W.w])
+    return {"value": round(aggregate(ops, world, t_max) / 1e12, 3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(t_max * 1e3 / args.steps, 4)}
+
+
+# ------------------------------------------------------- CPU oracle arm ----
+def oracle_sample_layers():
+    """A bounded sample of the workload for the CPU oracle: the M = 1 and
+    M = 16 rows of the step over all seven layers."""
+    from bit_group_quantized_flexq_b200 import inputs
+    return [1, 16], list(inputs.LLAMA2_7B_LAYERS)
+
+
+class OracleSample:
+    def __init__(self):
+        from bit_group_quantized_flexq_b200 import inputs
+        from oracle import flexq_oracle as orc
+        self.orc = orc
+        self.ms, self.layers = oracle_sample_layers()
+        self.w = []
+        for name, N, K in self.layers:
+            w16 = inputs.weights(N, K, std=0.02, seed=inputs.layer_seed("7b", name)).numpy()
+            qw, sw = orc.quantize_weight(w16, GS)      # offline step, not timed
+            self.w.append((name, N, K, qw, sw))
+        self.x = {(M, K): inputs.activations(M, K, outlier_frac=0.01, outlier_scale=20.0,
+                                             seed=inputs.layer_seed("7b-x", M, K)).numpy()
+                  for M in self.ms for K in {K for (_, _, K) in self.layers}}
+        self.ops = step_ops(self.ms, self.layers)
+
+    def step(self):
+        orc = self.orc
+        for M in self.ms:
+            for (name, N, K, qw, sw) in self.w:
+                qa, sa = orc.quantize_act(self.x[(M, K)], GS, ACT_BITS)
+                orc.to_fp16(orc.gemm_fp64(qa, sa, qw, sw, GS))
+
+
+def run_cpu_baseline(budget_s=20.0):
+    s = OracleSample()
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        s.step()
+        n += 1
+        if time.perf_counter() - t0 > budget_s / 2 or n >= 3:
+            break
+    dt = (time.perf_counter() - t0) / n
+    return {"value": round(s.ops / dt / 1e12, 9), "unit": UNIT, "cores": 1,
+            "kind": "oracle",
+            "sample": (f"oracle (numpy, int64 group dot products + FP64 rescale) on M in "
+                       f"{s.ms} over all seven LLaMA-2-7B layers; {n} passes of "
+                       f"{dt:.2f} s; integer matmul runs on one thread")}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    s = OracleSample()
+    for _ in range(args.warmup):
+        s.step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        s.step()
+    dt = time.perf_counter() - t0
+    value = s.ops * args.steps / dt / 1e12
+    ms, layers = workload_shapes()
+    out = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 9), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3 / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int64", "data": "synthetic",
+        "config": {"workload": workload_name(ms, layers),
+                   "sample": f"each step: M in {s.ms} over all seven layers"},
+        "cpu_baseline": {"value": round(value, 9), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"M in {s.ms} over all seven layers per step"},
+        "e2e": {"value": round(value, 9), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------------------ main ---
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["flexq", "reference"], default="flexq")
+    p.add_argument("--ms", type=lambda s: [int(v) for v in s.split(",")], default=None,
+                   help="subset of M values (profiling)")
+    p.add_argument("--layers", type=lambda s: s.split(","), default=None,
+                   help="subset of layer names (profiling)")
+    p.add_argument("--no-graph", dest="graph", action="store_false")
+    p.add_argument("--no-e2e", dest="e2e", action="store_false")
+    p.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    p.add_argument("--no-diag", dest="diag", action="store_false")
+    p.add_argument("--cpu-budget-s", type=float, default=20.0)
+    a = p.parse_args(argv)
+    if a.warmup < 3 and a.impl == "flexq" and not (a.ms or a.layers):
+        p.error("--warmup must be >= 3")
+    return a
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world = dist_init("nccl" if args.impl == "flexq" else "gloo")
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_flexq(args, rank, world)
+    finally:
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -242,6 +242,7 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
                 const void* Ws, void* Y, int32_t* P, bool partials, void* stream) {
   int rc = check_gemm_shape(M, N, K, gs);
   if (rc) return rc;
+  if (M == 0) return ok();               // empty batch: nothing to read or write
   if (partials) {
     const void* ptrs[] = {Xq, Wp, P};
     const char* names[] = {"Xq", "Wq_packed", "P"};
@@ -251,7 +252,6 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
     const char* names[] = {"Xq", "X_scales", "Wq_packed", "W_scales", "Y"};
     if ((rc = check_ptrs(5, ptrs, names))) return rc;
   }
-  if (M == 0) return ok();
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
   const Plan plan = make_plan(M, N, K, gs, st->sms, partials);
@@ -330,11 +330,11 @@ int flexq_quantize_act(int M, int K, int group_size, int bits, const void* X_fp1
   if (bits != 6 && bits != 8) return fail(FLEXQ_ERR_INVALID_ARG, "bits=%d is not 6 or 8", bits);
   if (!valid_gs(group_size)) return fail(FLEXQ_ERR_UNSUPPORTED, "group_size %d not in {32,64,128,256}", group_size);
   if (K % group_size) return fail(FLEXQ_ERR_UNSUPPORTED, "K=%d is not a multiple of group_size %d", K, group_size);
+  if (M == 0) return ok();               // empty batch: nothing to read or write
   const void* ptrs[] = {X_fp16, Xq, X_scales_fp16};
   const char* names[] = {"X_fp16", "Xq", "X_scales_fp16"};
   int rc = check_ptrs(3, ptrs, names);
   if (rc) return rc;
-  if (M == 0) return ok();
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
   const long long chunks = static_cast<long long>(M) * K / 8;

@@ -18,7 +18,8 @@
  *     channels, gs = group size along K, G = K / gs.
  *   - Supported shapes: M >= 0 (M == 0 is a no-op), N % 128 == 0, K % 128 == 0,
  *     gs in {32, 64, 128, 256}, K % gs == 0.
- *   - Every device pointer must be 16-byte aligned.
+ *   - Every device pointer must be 16-byte aligned.  With M == 0 the
+ *     activation-side pointers are not read and may be NULL.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
  *     are asynchronous: they validate their arguments, enqueue the work on
  *     `stream` and return.  Invalid arguments are reported before anything
