@@ -222,7 +222,8 @@ class Layers:
                                        seed=inputs.layer_seed("7b-x", M, K))
                 self.x[(M, K)] = x.to(device)
                 self.xq[(M, K)] = torch.empty(M, K, dtype=torch.int8, device=device)
-                self.xs[(M, K)] = torch.empty(M, K // GS, dtype=torch.float16, device=device)
+                self.xs[(M, K)] = torch.empty(K // GS, flexq.act_scales_ld(M),
+                                              dtype=torch.float16, device=device)
             for (name, N, K) in layers:
                 self.y[(M, name)] = torch.empty(M, N, dtype=torch.float16, device=device)
         torch.cuda.synchronize(device)
@@ -230,27 +231,39 @@ class Layers:
     def launches_per_step(self):
         return 2 * len(self.ms) * len(self.w)
 
-    def step(self, marks=None, gemm_marks=None, dominant_m=None):
-        """One pass of the hot path.  marks: events recorded at the start and
-        after each M group; gemm_marks: (start, end) events around each GEMM
-        of the dominant M."""
+    def quant(self, M, layer):
         from bit_group_quantized_flexq_b200 import flexq
-        gi = 0
-        if marks is not None:
-            marks[0].record()
-        for mi, M in enumerate(self.ms):
-            for (name, N, K, wp, ws) in self.w:
-                xq, xs = flexq.quantize_act(self.x[(M, K)], GS, ACT_BITS,
-                                            out=(self.xq[(M, K)], self.xs[(M, K)]))
-                timed = gemm_marks is not None and M == dominant_m
-                if timed:
-                    gemm_marks[gi][0].record()
-                flexq.gemm(xq, xs, wp, ws, N, GS, ACT_BITS, out=self.y[(M, name)])
-                if timed:
-                    gemm_marks[gi][1].record()
-                    gi += 1
-            if marks is not None:
-                marks[mi + 1].record()
+        _, _, K, _, _ = layer
+        flexq.quantize_act(self.x[(M, K)], GS, ACT_BITS, out=(self.xq[(M, K)], self.xs[(M, K)]))
+
+    def gemm(self, M, layer):
+        from bit_group_quantized_flexq_b200 import flexq
+        name, N, K, wp, ws = layer
+        flexq.gemm(self.xq[(M, K)], self.xs[(M, K)], wp, ws, N, GS, ACT_BITS,
+                   out=self.y[(M, name)])
+
+    def run_m(self, M):
+        for layer in self.w:
+            self.quant(M, layer)
+            self.gemm(M, layer)
+
+    def step(self):
+        for M in self.ms:
+            self.run_m(M)
+
+    def segments(self, dominant_m):
+        """The step cut into replayable pieces: all layers of an M as one piece,
+        except at the dominant M, where every quantization and every GEMM is
+        its own piece so that events can bracket the GEMM launches."""
+        segs = []
+        for M in self.ms:
+            if M == dominant_m:
+                for layer in self.w:
+                    segs.append(("quant", M, layer[0], (lambda M=M, l=layer: self.quant(M, l))))
+                    segs.append(("gemm", M, layer[0], (lambda M=M, l=layer: self.gemm(M, l))))
+            else:
+                segs.append(("all", M, None, (lambda M=M: self.run_m(M))))
+        return segs
 
 
 def run_flexq(args, rank, world):
@@ -266,53 +279,54 @@ def run_flexq(args, rank, world):
     ops = step_ops(ms, layers)
     nlay = len(layers)
 
-    def new_events(n):
-        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-
     # eager warm-up (first calls set kernel attributes; nothing is captured yet)
     for _ in range(2):
         W.step()
     torch.cuda.synchronize(device)
 
     stream = torch.cuda.Stream(device)
-    graphs, marks, gmarks = [], [], []
+    segs = W.segments(dominant_m)
+    runners = []
     if args.graph:
-        for i in range(args.steps):
-            mk = new_events(len(ms) + 1)
-            gm = [new_events(2) for _ in range(nlay)]
+        for (_, _, _, fn) in segs:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.stream(stream):
                 with torch.cuda.graph(g, stream=stream):
-                    W.step(mk, gm, dominant_m)
-            graphs.append(g)
-            marks.append(mk)
-            gmarks.append(gm)
+                    fn()
+            runners.append(g.replay)
+        graphs = runners
         torch.cuda.synchronize(device)
+    else:
+        runners = [fn for (_, _, _, fn) in segs]
+        graphs = []
 
-    def run_step(i):
-        if args.graph:
-            graphs[i].replay()
-        else:
-            W.step(marks[i], gmarks[i], dominant_m)
+    def new_event():
+        return torch.cuda.Event(enable_timing=True)
 
-    if not args.graph:
-        marks = [new_events(len(ms) + 1) for _ in range(args.steps)]
-        gmarks = [[new_events(2) for _ in range(nlay)] for _ in range(args.steps)]
+    # one event before the first piece and one after every piece, per step
+    evs = [[new_event() for _ in range(len(segs) + 1)] for _ in range(args.steps)]
+
+    def run_step(ev):
+        if ev is not None:
+            ev[0].record(stream)
+        for k, run in enumerate(runners):
+            run()
+            if ev is not None:
+                ev[k + 1].record(stream)
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            run_step(i % max(1, args.steps))
+            run_step(None)
         torch.cuda.synchronize(device)
         barrier(device)
         torch.cuda.synchronize(device)
         clocks = ClockSampler(device.index if device.index is not None else 0)
         clocks.start()
         time.sleep(0.3)                           # sampler up before timing
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
+        t0, t1 = new_event(), new_event()
         t0.record(stream)
         for i in range(args.steps):
-            run_step(i)
+            run_step(evs[i])
         t1.record(stream)
         torch.cuda.synchronize(device)
         clock_summary = clocks.stop()
@@ -323,11 +337,14 @@ def run_flexq(args, rank, world):
     if status != flexq.FLEXQ_OK:
         raise RuntimeError(f"device status after the timed region: {msg}")
 
-    # per-M time and dominant-kernel launches, from the events of the timed steps
-    per_m_ms = [statistics.mean(marks[i][mi].elapsed_time(marks[i][mi + 1])
-                                for i in range(args.steps)) for mi in range(len(ms))]
-    dom_durs = [gmarks[i][j][0].elapsed_time(gmarks[i][j][1])
-                for i in range(args.steps) for j in range(nlay)]
+    # per-M times and the dominant GEMM launches, from the timed steps' events
+    per_m_ms = []
+    for M in ms:
+        ks = [k for k, sg in enumerate(segs) if sg[1] == M]
+        per_m_ms.append(statistics.mean(evs[i][ks[0]].elapsed_time(evs[i][ks[-1] + 1])
+                                        for i in range(args.steps)))
+    gk = [k for k, sg in enumerate(segs) if sg[0] == "gemm"]
+    dom_durs = [evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps) for k in gk]
     dom_flops_per_step = sum(2.0 * dominant_m * N * K for (_, N, K) in layers)
     dom_avg_ms = statistics.mean(dom_durs)
     dom_flops_per_launch = dom_flops_per_step / nlay
@@ -388,6 +405,9 @@ def run_flexq(args, rank, world):
         "gpu_launches": W.launches_per_step() * args.steps,
         "clocks": clock_summary,
     }
+    if args.graph:
+        result["config"]["timing"] = ("CUDA-graph replay: one graph per M, one per launch at "
+                                      f"M={dominant_m}; events between graph launches")
     if diag:
         result["gemm_by_m"] = diag
     if args.e2e:
@@ -397,6 +417,7 @@ def run_flexq(args, rank, world):
     if rank == 0:
         print(json.dumps(result), flush=True)
     graphs.clear()
+    runners.clear()
 
 
 def gemm_diagnostics(W, device, hbm_gbs, int8_peak_tops, reps=10):

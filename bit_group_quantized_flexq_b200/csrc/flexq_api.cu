@@ -190,11 +190,32 @@ int encode_x_map(CUtensorMap* map, const void* xq, int M, int K, int T) {
   return FLEXQ_OK;
 }
 
+// FP16 scales stored group-major: [G rows][ld elements]; box = `box_rows`
+// consecutive elements (tokens or weight rows) x 8 groups; elements past
+// `extent` and groups past G read as zero.
+int encode_scale_map(CUtensorMap* map, const void* scales, int extent, int ld, int G,
+                     int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(FLEXQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(extent), static_cast<cuuint64_t>(G)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_rows), 8u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(scales), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(FLEXQ_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", static_cast<int>(r));
+  return FLEXQ_OK;
+}
+
+int act_scales_ld(int M) { return (M + 7) / 8 * 8; }
+
 // --------------------------------------------------------------- launches --
 template <int T>
 int ctrl_offset_for(int split) {
   using Cfg = flexq::GemmCfg<T>;
-  int stage = Cfg::kStages * Cfg::kStageBytes;
+  int stage = Cfg::kMainBytes;
   int red = (split - 1) * 128 * T * 4;
   int off = stage > red ? stage : red;
   return (off + 15) & ~15;
@@ -206,7 +227,8 @@ int smem_bytes_for(int split) {
 }
 
 template <int T, bool PARTIALS>
-int launch_gemm_t(DeviceState* st, const CUtensorMap& map, flexq::GemmArgs a, cudaStream_t stream) {
+int launch_gemm_t(DeviceState* st, const CUtensorMap& map, const CUtensorMap& map_sa,
+                  const CUtensorMap& map_sw, flexq::GemmArgs a, cudaStream_t stream) {
   using Cfg = flexq::GemmCfg<T>;
   auto kern = flexq::gemm_w6ax_kernel<T, PARTIALS>;
   const unsigned bit = 1u << ((T == 16 ? 0 : T == 32 ? 1 : T == 64 ? 2 : 3) + (PARTIALS ? 4 : 0));
@@ -233,7 +255,7 @@ int launch_gemm_t(DeviceState* st, const CUtensorMap& map, flexq::GemmArgs a, cu
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = a.split > 1 ? 1 : 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map, map_sa, map_sw, a);
   if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
   return FLEXQ_OK;
 }
@@ -255,12 +277,17 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
   const Plan plan = make_plan(M, N, K, gs, st->sms, partials);
-  CUtensorMap map;
+  CUtensorMap map, map_sa, map_sw;
   if ((rc = encode_x_map(&map, Xq, M, K, plan.T))) return rc;
+  memset(&map_sa, 0, sizeof(map_sa));
+  memset(&map_sw, 0, sizeof(map_sw));
+  if (!partials) {
+    const int G = K / gs;
+    if ((rc = encode_scale_map(&map_sa, Xs, M, act_scales_ld(M), G, plan.T))) return rc;
+    if ((rc = encode_scale_map(&map_sw, Ws, N, N, G, 128))) return rc;
+  }
   flexq::GemmArgs a = {};
-  a.xs = static_cast<const __half*>(Xs);
   a.wp = static_cast<const uint8_t*>(Wp);
-  a.ws = static_cast<const __half*>(Ws);
   a.y = static_cast<__half*>(Y);
   a.p = P;
   a.status = st->status;
@@ -269,10 +296,10 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
   a.stall = g_inject_stall.exchange(0);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (plan.T) {
-    case 16: rc = partials ? launch_gemm_t<16, true>(st, map, a, s) : launch_gemm_t<16, false>(st, map, a, s); break;
-    case 32: rc = partials ? launch_gemm_t<32, true>(st, map, a, s) : launch_gemm_t<32, false>(st, map, a, s); break;
-    case 64: rc = partials ? launch_gemm_t<64, true>(st, map, a, s) : launch_gemm_t<64, false>(st, map, a, s); break;
-    default: rc = partials ? launch_gemm_t<128, true>(st, map, a, s) : launch_gemm_t<128, false>(st, map, a, s); break;
+    case 16: rc = partials ? launch_gemm_t<16, true>(st, map, map_sa, map_sw, a, s) : launch_gemm_t<16, false>(st, map, map_sa, map_sw, a, s); break;
+    case 32: rc = partials ? launch_gemm_t<32, true>(st, map, map_sa, map_sw, a, s) : launch_gemm_t<32, false>(st, map, map_sa, map_sw, a, s); break;
+    case 64: rc = partials ? launch_gemm_t<64, true>(st, map, map_sa, map_sw, a, s) : launch_gemm_t<64, false>(st, map, map_sa, map_sw, a, s); break;
+    default: rc = partials ? launch_gemm_t<128, true>(st, map, map_sa, map_sw, a, s) : launch_gemm_t<128, false>(st, map, map_sa, map_sw, a, s); break;
   }
   return rc ? rc : ok();
 }
@@ -295,6 +322,8 @@ const char* flexq_status_string(int status) {
 }
 
 const char* flexq_last_error_message(void) { return t_last_error.c_str(); }
+
+size_t flexq_act_scales_ld(int M) { return M > 0 ? static_cast<size_t>(act_scales_ld(M)) : 0; }
 
 size_t flexq_weight_packed_bytes(int N, int K, int group_size) {
   if (N <= 0 || K <= 0 || N % 128 || K % 128 || !valid_gs(group_size) || K % group_size) return 0;
@@ -347,11 +376,12 @@ int flexq_quantize_act(int M, int K, int group_size, int bits, const void* X_fp1
   uint2* q = reinterpret_cast<uint2*>(Xq);
   __half* xs = static_cast<__half*>(X_scales_fp16);
   const int cpr = K / 8;
+  const int ld = act_scales_ld(M);
   switch (group_size) {
-    case 32: flexq::quant_act_kernel<32><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, qmax); break;
-    case 64: flexq::quant_act_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, qmax); break;
-    case 128: flexq::quant_act_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, qmax); break;
-    default: flexq::quant_act_kernel<256><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, qmax); break;
+    case 32: flexq::quant_act_kernel<32><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, ld, qmax); break;
+    case 64: flexq::quant_act_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, ld, qmax); break;
+    case 128: flexq::quant_act_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, ld, qmax); break;
+    default: flexq::quant_act_kernel<256><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, ld, qmax); break;
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "quant_act_kernel launch");

@@ -46,9 +46,7 @@ constexpr int kASlots = 4;            // TMEM A ring depth
 constexpr int kStatusTimeout = 5;     // == FLEXQ_ERR_DEVICE_TIMEOUT
 
 struct GemmArgs {
-  const __half* xs;        // [M, G] activation scales
   const uint8_t* wp;       // packed weights, device form
-  const __half* ws;        // [N, G] weight scales
   __half* y;               // [M, N] output (GEMM mode)
   int32_t* p;              // [G, M, N] partials (debug mode)
   unsigned int* status;    // device status word [4]
@@ -63,11 +61,18 @@ struct GemmCfg {
   static constexpr int kEpiWarps = (T <= 32) ? 4 : 8;
   static constexpr int kThreads = (6 + kEpiWarps) * 32;
   static constexpr int kCols = T / (kEpiWarps / 4);      // tokens per epi warp
-  static constexpr int kStages = (T == 16) ? 7 : (T == 32) ? 6 : (T == 64) ? 5 : 4;
+  static constexpr int kStages = (T == 16) ? 6 : (T == 32) ? 5 : 4;
   static constexpr int kMinBlocks = (T <= 64) ? 2 : 1;
   static constexpr int kMaxSplit = (T == 16) ? 8 : (T == 32) ? 6 : (T == 64) ? 4 : 2;
   static constexpr int kXsBytes = T * 128;
   static constexpr int kStageBytes = kXsBytes + kWTileBytes;
+  // scale ring: one slot holds 8 groups ("octet") of activation scales for
+  // the T tokens ([8][T] fp16) and of weight scales for the 128 rows
+  // ([8][128] fp16), each brought by one TMA box
+  static constexpr int kScSlots = 3;
+  static constexpr int kScSaBytes = 8 * T * 2;
+  static constexpr int kScSlotBytes = kScSaBytes + 8 * 128 * 2;
+  static constexpr int kMainBytes = kStages * kStageBytes + kScSlots * kScSlotBytes;
   static constexpr int kPCol0 = 0;
   static constexpr int kACol0 = 2 * T;
   static constexpr int kTmemCols = (2 * T + 128 <= 256) ? 256 : 512;
@@ -83,10 +88,13 @@ struct GemmCtrl {
   uint64_t a_empty[kASlots];
   uint64_t p_full[2];
   uint64_t p_empty[2];
+  uint64_t s_full[GemmCfg<T>::kScSlots];
+  uint64_t s_empty[GemmCfg<T>::kScSlots];
   uint64_t done;
   uint32_t tmem_base;
   uint32_t pad;
-  float sa[GemmCfg<T>::kEpiWarps][GemmCfg<T>::kCols];
+  // per epilogue warp: its tokens' activation scales of the current octet, FP32
+  float sa[GemmCfg<T>::kEpiWarps][8][GemmCfg<T>::kCols];
 };
 
 __device__ __forceinline__ void record_status(unsigned int* status, int code,
@@ -137,13 +145,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 
 template <int T, bool PARTIALS>
 __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
-    gemm_w6ax_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
+    gemm_w6ax_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                     const __grid_constant__ CUtensorMap tmap_sa,
+                     const __grid_constant__ CUtensorMap tmap_sw, const GemmArgs args) {
   using Cfg = GemmCfg<T>;
   constexpr int STAGES = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* xs_ring = base;                                  // STAGES * kXsBytes
   uint8_t* w_ring = base + STAGES * Cfg::kXsBytes;          // STAGES * 12288
+  uint8_t* sc_ring = w_ring + STAGES * kWTileBytes;         // kScSlots slots
   float* red = reinterpret_cast<float*>(base);              // cluster reduction
   GemmCtrl<T>* ctrl = reinterpret_cast<GemmCtrl<T>*>(base + args.ctrl_offset);
 
@@ -162,7 +173,6 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   const int u1 = static_cast<int>((static_cast<long long>(ks + 1) * units) / S);
   const int kb0 = u0 * U;
   const int nkb = (u1 - u0) * U;
-  const int G = K / gs;
   const int g0 = kb0 * kKBlock / gs;
   const int ngroups = nkb * kKBlock / gs;
 
@@ -179,9 +189,17 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       mbar_init(&ctrl->p_full[b], 1);
       mbar_init(&ctrl->p_empty[b], Cfg::kEpiWarps);
     }
+    for (int s = 0; s < Cfg::kScSlots; ++s) {
+      mbar_init(&ctrl->s_full[s], 1);
+      mbar_init(&ctrl->s_empty[s], Cfg::kEpiWarps);
+    }
     mbar_init(&ctrl->done, 1);
     fence_barrier_init();
     prefetch_tensormap(&tmap_x);
+    if (!PARTIALS) {
+      prefetch_tensormap(&tmap_sa);
+      prefetch_tensormap(&tmap_sw);
+    }
   }
   if (warp == 1) tmem_alloc(&ctrl->tmem_base, Cfg::kTmemCols);
   tc_fence_before();
@@ -197,9 +215,31 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   if (warp == 0) {
     // ------------------------------------------------------- producer ----
     if (lane == 0) {
-      uint32_t issued = 0, parity = 0;
+      uint32_t issued = 0, parity = 0, sc_issued = 0, sc_parity = 0;
+      const int n_oct = PARTIALS ? 0 : (ngroups + 7) / 8;
+      int next_oct = 0;
       bool ok = true;
-      for (int i = 0; i < nkb; ++i) {
+      for (int i = 0; i < nkb && ok; ++i) {
+        // scales: issue octet o at the first K block that touches group 8*o
+        const int lg_first = i * kKBlock / gs;
+        while (next_oct < n_oct && next_oct * 8 <= lg_first) {
+          const int o = next_oct, slot = o % Cfg::kScSlots;
+          if (o >= Cfg::kScSlots &&
+              !mbar_wait(&ctrl->s_empty[slot], ((o / Cfg::kScSlots) - 1) & 1, lim)) {
+            ok = false;
+            break;
+          }
+          uint8_t* dst = sc_ring + slot * Cfg::kScSlotBytes;
+          mbar_arrive_expect_tx(&ctrl->s_full[slot], Cfg::kScSlotBytes);
+          tma_load_2d(dst, &tmap_sa, &ctrl->s_full[slot], mt * T, g0 + 8 * o);
+          tma_load_2d(dst + Cfg::kScSaBytes, &tmap_sw, &ctrl->s_full[slot], nt * kTileRows,
+                      g0 + 8 * o);
+          sc_issued |= 1u << slot;
+          sc_parity = (sc_parity & ~(1u << slot)) |
+                      (static_cast<uint32_t>((o / Cfg::kScSlots) & 1) << slot);
+          ++next_oct;
+        }
+        if (!ok) break;
         const int s = i % STAGES;
         if (i >= STAGES &&
             !mbar_wait(&ctrl->empty[s], ((i / STAGES) - 1) & 1, lim)) {
@@ -220,6 +260,8 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       // every issued copy must land before the CTA may finish
       for (int s = 0; s < STAGES; ++s)
         if ((issued >> s) & 1u) mbar_wait(&ctrl->full[s], (parity >> s) & 1u, lim);
+      for (int s = 0; s < Cfg::kScSlots; ++s)
+        if ((sc_issued >> s) & 1u) mbar_wait(&ctrl->s_full[s], (sc_parity >> s) & 1u, lim);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -319,42 +361,34 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     const int n = nt * kTileRows + row;
     const int col0 = c * Cfg::kCols;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    float* sa_w = ctrl->sa[e];
     const int m_base = mt * T + col0;
-    // activation scales of this warp's tokens for a group: lane l holds
-    // tokens col0 + l and col0 + l + 32
-    auto load_sa = [&](int g, float (&v)[2]) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int t = lane + 32 * h;
-        const int m = m_base + t;
-        v[h] = (t < Cfg::kCols && m < M)
-                   ? __half2float(args.xs[static_cast<size_t>(m) * G + g])
-                   : 0.0f;
-      }
-    };
-    float sa_next[2] = {0.0f, 0.0f};
-    float sw_next = 0.0f;
-    if (ngroups > 0) {
-      if (!PARTIALS) load_sa(g0, sa_next);
-      if (!PARTIALS) sw_next = __half2float(args.ws[static_cast<size_t>(n) * G + g0]);
-    }
     for (int lg = 0; lg < ngroups; ++lg) {
       const int b = lg & 1;
       const int g = g0 + lg;
+      const int gi = lg & 7;
+      const int sc_slot = (lg >> 3) % Cfg::kScSlots;
+      const uint8_t* sc = sc_ring + sc_slot * Cfg::kScSlotBytes;
       float swn = 0.0f;
       if (!PARTIALS) {
-        __syncwarp();
+        if (gi == 0) {
+          if (!warp_wait(&ctrl->s_full[sc_slot], ((lg >> 3) / Cfg::kScSlots) & 1, lim)) {
+            if (lane == 0) record_status(args.status, kStatusTimeout, 5);
+            break;
+          }
+          // this warp's tokens of the octet, FP16 -> FP32, into its own buffer
+          const __half* sa_h = reinterpret_cast<const __half*>(sc);
+          __syncwarp();
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-          if (lane + 32 * h < Cfg::kCols) sa_w[lane + 32 * h] = sa_next[h];
-        __syncwarp();
-        swn = sw_next * 0.25f;               // codes in TMEM are 4 * code
-        if (lg + 1 < ngroups) {
-          load_sa(g + 1, sa_next);
-          sw_next = __half2float(args.ws[static_cast<size_t>(n) * G + g + 1]);
+          for (int idx = lane; idx < 8 * Cfg::kCols; idx += 32) {
+            const int gg = idx / Cfg::kCols, j = idx - gg * Cfg::kCols;
+            ctrl->sa[e][gg][j] = __half2float(sa_h[gg * T + col0 + j]);
+          }
+          __syncwarp();
         }
+        const __half* sw_h = reinterpret_cast<const __half*>(sc + Cfg::kScSaBytes);
+        swn = __half2float(sw_h[gi * kTileRows + row]) * 0.25f;   // TMEM holds 4 * code
       }
+      const float* sa_w = ctrl->sa[e][gi];
       if (!warp_wait(&ctrl->p_full[b], (lg >> 1) & 1, lim)) {
         if (lane == 0) record_status(args.status, kStatusTimeout, 4);
         break;
@@ -391,6 +425,10 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
             acc[ch * CH + j] = fmaf(static_cast<float>(static_cast<int32_t>(pv[j])),
                                     swn * sa_w[ch * CH + j], acc[ch * CH + j]);
         }
+      }
+      if (!PARTIALS && (gi == 7 || lg == ngroups - 1)) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->s_empty[sc_slot]);
       }
     }
   }

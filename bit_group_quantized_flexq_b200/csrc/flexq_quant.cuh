@@ -6,6 +6,9 @@
 // Scale rule: s = fp16_rne(absmax / Q) with an IEEE FP32 division; codes =
 // clamp(round_half_even(x / s), -Q, Q) with an IEEE FP32 division by the
 // stored FP16 scale; a zero FP16 scale gives zero codes.
+//
+// Scales are stored group-major (scale of row r, group g at g * ld + r) so
+// that the GEMM can fetch eight groups of a tile's scales with one TMA box.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -32,7 +35,7 @@ __device__ __forceinline__ int quant_code(float x, float s, int qmax) {
 template <int GS>
 __global__ void __launch_bounds__(256) quant_act_kernel(
     const uint4* __restrict__ X, uint2* __restrict__ Xq, __half* __restrict__ Xs,
-    long long chunks, int chunks_per_row, int qmax) {
+    long long chunks, int chunks_per_row, int ld_scales, int qmax) {
   constexpr int LANES = GS / 8;            // lanes per group
   static_assert(LANES >= 4 && LANES <= 32, "group size 32..256");
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
@@ -72,25 +75,22 @@ __global__ void __launch_bounds__(256) quant_act_kernel(
       Xq[idx] = make_uint2(lo, hi);
       const long long row = idx / chunks_per_row;
       const int c = static_cast<int>(idx - row * chunks_per_row);
-      if ((c % LANES) == 0) {
-        const int G = chunks_per_row / LANES;
-        Xs[row * G + c / LANES] = s16;
-      }
+      if ((c % LANES) == 0) Xs[static_cast<long long>(c / LANES) * ld_scales + row] = s16;
     }
   }
 }
 
 // --------------------------------------------------------------------------
 // Weight quantization, pass 1: one thread per (row n, group g) computes the
-// group's FP16 scale.
+// group's FP16 scale, stored at Ws[g * N + n].
 // --------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) weight_scale_kernel(
     const __half* __restrict__ W, __half* __restrict__ Ws, int N, int K, int gs) {
   const int G = K / gs;
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= static_cast<long long>(N) * G) return;
-  const int n = static_cast<int>(t / G);
-  const int g = static_cast<int>(t - static_cast<long long>(n) * G);
+  const int g = static_cast<int>(t / N);
+  const int n = static_cast<int>(t - static_cast<long long>(g) * N);
   const uint4* p = reinterpret_cast<const uint4*>(W + static_cast<long long>(n) * K + g * gs);
   float amax = 0.0f;
   for (int c = 0; c < gs / 8; ++c) {
@@ -124,7 +124,6 @@ __global__ void __launch_bounds__(256) weight_pack_kernel(
   const int n = static_cast<int>(nk / KB);
   const int kb = static_cast<int>(nk - static_cast<long long>(n) * KB);
   const int k0 = kb * 128 + half_idx * 64;
-  const int G = K / gs;
   const uint4* p = reinterpret_cast<const uint4*>(W + static_cast<long long>(n) * K + k0);
   uint32_t word[12];
 #pragma unroll
@@ -134,7 +133,7 @@ __global__ void __launch_bounds__(256) weight_pack_kernel(
     uint4 raw = __ldg(p + c);
     const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
     const int kk = k0 + c * 8;
-    const float s = __half2float(Ws[static_cast<long long>(n) * G + kk / gs]);
+    const float s = __half2float(Ws[static_cast<long long>(kk / gs) * N + n]);
     uint32_t u[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {

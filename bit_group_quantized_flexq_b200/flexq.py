@@ -44,6 +44,7 @@ def lib():
             "flexq_status_string": (ctypes.c_char_p, [c_int]),
             "flexq_last_error_message": (ctypes.c_char_p, []),
             "flexq_weight_packed_bytes": (c_size_t, [c_int, c_int, c_int]),
+            "flexq_act_scales_ld": (c_size_t, [c_int]),
             "flexq_quantize_weight": (c_int, [c_int, c_int, c_int, c_void_p, c_void_p,
                                               c_void_p, c_void_p]),
             "flexq_quantize_act": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p,
@@ -104,8 +105,23 @@ def weight_packed_bytes(N, K, group_size):
     return int(lib().flexq_weight_packed_bytes(N, K, group_size))
 
 
+def act_scales_ld(M):
+    return int(lib().flexq_act_scales_ld(M))
+
+
+def act_scales_view(xs, M):
+    """The [M, G] view of group-major activation scales ([G, ld] storage)."""
+    return xs[:, :M].t()
+
+
+def weight_scales_view(ws):
+    """The [N, G] view of group-major weight scales ([G, N] storage)."""
+    return ws.t()
+
+
 def quantize_weight(w, group_size, out=None):
-    """FP16 W [N, K] -> (packed uint8 [3NK/4] in the device form, FP16 scales [N, K/gs])."""
+    """FP16 W [N, K] -> (packed uint8 [3NK/4] in the device form, FP16 scales
+    stored group-major as a [K/gs, N] tensor)."""
     _need(w, "w", torch.float16)
     N, K = w.shape
     nbytes = weight_packed_bytes(N, K, group_size)
@@ -113,24 +129,26 @@ def quantize_weight(w, group_size, out=None):
         raise FlexQError(FLEXQ_ERR_UNSUPPORTED, f"unsupported weight shape {N}x{K}, gs={group_size}")
     if out is None:
         out = (torch.empty(nbytes, dtype=torch.uint8, device=w.device),
-               torch.empty(N, K // group_size, dtype=torch.float16, device=w.device))
+               torch.empty(K // group_size, N, dtype=torch.float16, device=w.device))
     wp, ws = out
     _need(wp, "packed", torch.uint8, (nbytes,))
-    _need(ws, "scales", torch.float16, (N, K // group_size))
+    _need(ws, "scales", torch.float16, (K // group_size, N))
     _check(lib().flexq_quantize_weight(N, K, group_size, _ptr(w), _ptr(wp), _ptr(ws), _stream(w)))
     return wp, ws
 
 
 def quantize_act(x, group_size, bits, out=None):
-    """FP16 X [M, K] -> (int8 codes [M, K], FP16 scales [M, K/gs])."""
+    """FP16 X [M, K] -> (int8 codes [M, K], FP16 scales stored group-major as a
+    [K/gs, act_scales_ld(M)] tensor; see act_scales_view)."""
     _need(x, "x", torch.float16)
     M, K = x.shape
+    ld = act_scales_ld(M)
     if out is None:
         out = (torch.empty(M, K, dtype=torch.int8, device=x.device),
-               torch.empty(M, K // group_size, dtype=torch.float16, device=x.device))
+               torch.empty(K // group_size, ld, dtype=torch.float16, device=x.device))
     xq, xs = out
     _need(xq, "codes", torch.int8, (M, K))
-    _need(xs, "scales", torch.float16, (M, K // group_size))
+    _need(xs, "scales", torch.float16, (K // group_size, ld))
     _check(lib().flexq_quantize_act(M, K, group_size, bits, _ptr(x), _ptr(xq), _ptr(xs), _stream(x)))
     return xq, xs
 
@@ -139,9 +157,9 @@ def gemm(xq, xs, wp, ws, N, group_size, act_bits=6, out=None):
     """Y [M, N] FP16 = dequant(xq, xs) . dequant(wp, ws)^T (W6A6 or W6A8)."""
     _need(xq, "xq", torch.int8)
     M, K = xq.shape
-    _need(xs, "xs", torch.float16, (M, K // group_size))
+    _need(xs, "xs", torch.float16, (K // group_size, act_scales_ld(M)))
     _need(wp, "wp", torch.uint8, (weight_packed_bytes(N, K, group_size),))
-    _need(ws, "ws", torch.float16, (N, K // group_size))
+    _need(ws, "ws", torch.float16, (K // group_size, N))
     if out is None:
         out = torch.empty(M, N, dtype=torch.float16, device=xq.device)
     _need(out, "out", torch.float16, (M, N))

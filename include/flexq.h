@@ -56,6 +56,13 @@ const char* flexq_status_string(int status);
 const char* flexq_last_error_message(void);
 
 /*
+ * Leading dimension (in elements) of the group-major activation scales for a
+ * batch of M tokens: M rounded up to a multiple of 8, so that every group's
+ * row starts on a 16-byte boundary.  0 for M <= 0.
+ */
+size_t flexq_act_scales_ld(int M);
+
+/*
  * Size in bytes of the packed 6-bit weight buffer for an [N, K] layer:
  * 3*N*K/4 (four codes in three bytes).  Returns 0 for unsupported shapes.
  */
@@ -77,8 +84,9 @@ size_t flexq_weight_packed_bytes(int N, int K, int group_size);
  *                 tile, byte b of 16-byte chunk j (0..5) of row r holds
  *                 canonical byte kb*96 + 16*j + b of row nt*128 + r and sits
  *                 at offset (j*128 + r)*16 + b.
- *   W_scales_fp16 out, [N, G] FP16: s = fp16_rne(absmax / 31) per (n, group),
- *                 absmax/31 computed as an IEEE FP32 division.
+ *   W_scales_fp16 out, N*G FP16 values stored group-major: the scale of row
+ *                 n, group g is element g*N + n.  s = fp16_rne(absmax / 31)
+ *                 with absmax/31 computed as an IEEE FP32 division.
  * Codes: clamp(round_half_even(w / s), -31, 31) with an IEEE FP32 division by
  * the stored FP16 scale; a group whose FP16 scale is 0 gets all-zero codes.
  */
@@ -94,7 +102,11 @@ int flexq_quantize_weight(int N, int K, int group_size, const void* W_fp16,
  *   bits          6 (codes in [-31, 31], Q = 31) or 8 (codes in [-127, 127],
  *                 Q = 127).
  *   Xq            out, [M, K] int8, one code per byte for both widths.
- *   X_scales_fp16 out, [M, G] FP16: fp16_rne(absmax / Q) per (m, group).
+ *   X_scales_fp16 out, G * flexq_act_scales_ld(M) FP16 values stored
+ *                 group-major: the scale of token m, group g is element
+ *                 g*ld + m with ld = flexq_act_scales_ld(M) (M rounded up to
+ *                 a multiple of 8); entries m >= M are not written.
+ *                 s = fp16_rne(absmax / Q).
  * Same rounding rules as flexq_quantize_weight.
  */
 int flexq_quantize_act(int M, int K, int group_size, int bits,
@@ -107,9 +119,11 @@ int flexq_quantize_act(int M, int K, int group_size, int bits,
  * and recombined with the scales, dequantization fused into the GEMM (arXiv
  * abstract; blog, "Bridging Software and Hardware with BTC").
  *
- *   Xq, X_scales     activation codes [M, K] int8 and FP16 scales [M, G].
+ *   Xq, X_scales     activation codes [M, K] int8 and FP16 scales in the
+ *                    group-major layout of flexq_quantize_act.
  *   Wq_packed,       weight codes in the device form above and FP16 scales
- *   W_scales         [N, G], as written by flexq_quantize_weight.
+ *   W_scales         (group-major, g*N + n), as written by
+ *                    flexq_quantize_weight.
  *   Y_fp16           out, [M, N] FP16.
  * For each group g the integer partial P_g[m,n] = sum_{k in g} Xq[m,k]*Wq[n,k]
  * is formed exactly (int32), then Y[m,n] = fp16_rne(sum_g P_g[m,n] *

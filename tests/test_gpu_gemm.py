@@ -112,7 +112,7 @@ def test_gemm_empty_m_is_noop():
     w = inputs.weights(N, K, seed=3)
     wp, ws = flexq.quantize_weight(w.cuda(), gs)
     xq = torch.empty(0, K, dtype=torch.int8, device="cuda")
-    xs = torch.empty(0, K // gs, dtype=torch.float16, device="cuda")
+    xs = torch.empty(K // gs, 0, dtype=torch.float16, device="cuda")
     y = flexq.gemm(xq, xs, wp, ws, N, gs)
     assert y.shape == (0, N)
 
