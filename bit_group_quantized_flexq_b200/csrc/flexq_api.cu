@@ -461,4 +461,27 @@ int flexq_get_device_status(void* stream) {
               h[1] < 5 ? roles[h[1]] : "?", h[2]);
 }
 
+#ifdef FLEXQ_TRACE
+// Trace builds only: copies the pipeline trace of the last GEMM launch.
+int flexq_debug_read_trace(long long* host, size_t count) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  const size_t n = sizeof(flexq::g_flexq_trace) / sizeof(long long);
+  e = cudaMemcpyFromSymbol(host, flexq::g_flexq_trace, (count < n ? count : n) * sizeof(long long));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the trace");
+  return ok();
+}
+
+// Trace builds only: copies the per-CTA timeline ([cta][8]) of the last launch.
+int flexq_debug_read_cta_times(unsigned long long* host, size_t count) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  const size_t n = sizeof(flexq::g_flexq_cta_times) / sizeof(unsigned long long);
+  e = cudaMemcpyFromSymbol(host, flexq::g_flexq_cta_times,
+                           (count < n ? count : n) * sizeof(unsigned long long));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the CTA timeline");
+  return ok();
+}
+#endif
+
 }  // extern "C"

@@ -97,6 +97,38 @@ struct GemmCtrl {
   float sa[GemmCfg<T>::kEpiWarps][8][GemmCfg<T>::kCols];
 };
 
+// Optional pipeline trace (compile with -DFLEXQ_TRACE): CTA (0,0,0) records
+// clock64() offsets at fixed points of each role, [role][event][index], and
+// every CTA records %globaltimer at entry (0), after set-up (1), after its
+// roles' loops (2), at exit (3), after the TMEM release (5), after the first
+// cluster barrier (6) and before the output store (7); its SM id in slot 4.
+#ifdef FLEXQ_TRACE
+__device__ long long g_flexq_trace[4][4][1024];
+__device__ unsigned long long g_flexq_cta_times[8192][8];
+#define FLEXQ_TRACE_POINT(role, ev, idx, t0)                                   \
+  do {                                                                         \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (idx) < 1024) \
+      g_flexq_trace[role][ev][idx] = clock64() - (t0);                         \
+  } while (0)
+#define FLEXQ_CTA_TIME(slot)                                                   \
+  do {                                                                         \
+    const unsigned cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
+    if (threadIdx.x == 0 && cta_ < 8192) {                                     \
+      g_flexq_cta_times[cta_][slot] = global_timer_ns();                       \
+      unsigned smid_;                                                          \
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid_));                       \
+      g_flexq_cta_times[cta_][4] = smid_;                                      \
+    }                                                                          \
+  } while (0)
+#else
+#define FLEXQ_TRACE_POINT(role, ev, idx, t0) \
+  do {                                       \
+  } while (0)
+#define FLEXQ_CTA_TIME(slot) \
+  do {                       \
+  } while (0)
+#endif
+
 __device__ __forceinline__ void record_status(unsigned int* status, int code,
                                               int where) {
   if (atomicCAS(status, 0u, static_cast<unsigned>(code)) == 0u) {
@@ -105,11 +137,16 @@ __device__ __forceinline__ void record_status(unsigned int* status, int code,
   }
 }
 
-// All lanes wait; the warp agrees on the outcome.
+// Lane 0 waits (the other lanes park at the warp barrier instead of polling
+// the mbarrier); the warp agrees on the outcome.  The warp barrier orders the
+// waiting lane's acquire before every lane's subsequent reads.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
                                           uint64_t limit) {
-  const bool ok = mbar_wait(bar, parity, limit);
-  return __all_sync(0xffffffffu, ok);
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, limit);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
+  return ok;
 }
 
 // Four 6-bit codes in the low 24 bits of q (bits above 23 ignored) -> four
@@ -161,6 +198,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint64_t lim = args.wait_limit_ns;
+  FLEXQ_CTA_TIME(0);
 
   const int ks = blockIdx.x;            // K split index == rank in cluster
   const int nt = blockIdx.y;            // weight tile
@@ -206,6 +244,9 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
+  const long long t_start = clock64();
+  (void)t_start;
+  FLEXQ_CTA_TIME(1);
 
   // epilogue state lives across the role switch below
   float acc[Cfg::kCols];
@@ -255,6 +296,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
                   kWTileBytes, &ctrl->full[s]);
         issued |= 1u << s;
         parity = (parity & ~(1u << s)) | (static_cast<uint32_t>((i / STAGES) & 1) << s);
+        FLEXQ_TRACE_POINT(0, 0, i, t_start);
       }
       if (!ok) record_status(args.status, kStatusTimeout, 0);
       // every issued copy must land before the CTA may finish
@@ -279,6 +321,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
           break;
         }
         tc_fence_after();
+        FLEXQ_TRACE_POINT(1, 0, i, t_start);
         const uint32_t xs_addr = smem_u32(xs_ring + s * Cfg::kXsBytes);
 #pragma unroll
         for (int sub = 0; sub < 4; ++sub) {
@@ -293,6 +336,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
             }
             tc_fence_after();
           }
+          if (first) FLEXQ_TRACE_POINT(1, 1, lg, t_start);
           mma_i8_tmem_a(tmem + Cfg::kPCol0 + b * T,
                         tmem + Cfg::kACol0 + slot * 32 + sub * 8,
                         smem_desc_k_sw128(xs_addr + sub * 32), idesc,
@@ -305,6 +349,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         if (!ok) break;
         mma_commit(&ctrl->empty[s]);
         mma_commit(&ctrl->a_empty[slot]);
+        FLEXQ_TRACE_POINT(1, 2, i, t_start);
       }
       if (!ok) record_status(args.status, kStatusTimeout, 1);
       // all issued MMAs must finish before TMEM is released
@@ -323,6 +368,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         if (lane == 0) record_status(args.status, kStatusTimeout, 2);
         break;
       }
+      if (q == 0 && lane == 0) FLEXQ_TRACE_POINT(2, 0, i, t_start);
       const uint4* src = reinterpret_cast<const uint4*>(w_ring + s * kWTileBytes) + row;
       uint32_t wa[12], wb[12];
 #pragma unroll
@@ -341,6 +387,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         break;
       }
       tc_fence_after();
+      if (q == 0 && lane == 0) FLEXQ_TRACE_POINT(2, 1, i, t_start);
       const uint32_t col = tmem + lane_base + Cfg::kACol0 + slot * 32;
       uint32_t out[16];
       unpack48(wa, out);
@@ -351,6 +398,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->a_full[slot]);
+      if (q == 0 && lane == 0) FLEXQ_TRACE_POINT(2, 2, i, t_start);
     }
   } else {
     // ------------------------------------------------------ epilogue -----
@@ -375,6 +423,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
             if (lane == 0) record_status(args.status, kStatusTimeout, 5);
             break;
           }
+          if (e == 0 && lane == 0) FLEXQ_TRACE_POINT(3, 0, lg >> 3, t_start);
           // this warp's tokens of the octet, FP16 -> FP32, into its own buffer
           const __half* sa_h = reinterpret_cast<const __half*>(sc);
           __syncwarp();
@@ -394,6 +443,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         break;
       }
       tc_fence_after();
+      if (e == 0 && lane == 0) FLEXQ_TRACE_POINT(3, 1, lg, t_start);
       // drain the partials in chunks; the buffer is released right after the
       // last chunk has been read, before that chunk's arithmetic
       constexpr int CH = Cfg::kLdChunk;
@@ -410,6 +460,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctrl->p_empty[b]);
+          if (e == 0 && lane == 0) FLEXQ_TRACE_POINT(3, 2, lg, t_start);
         }
         if (PARTIALS) {
 #pragma unroll
@@ -426,6 +477,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
                                     swn * sa_w[ch * CH + j], acc[ch * CH + j]);
         }
       }
+      if (e == 0 && lane == 0) FLEXQ_TRACE_POINT(3, 3, lg, t_start);
       if (!PARTIALS && (gi == 7 || lg == ngroups - 1)) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->s_empty[sc_slot]);
@@ -436,11 +488,16 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   // ------------------------------------------------------------ teardown --
   tc_fence_before();
   __syncthreads();
+  FLEXQ_CTA_TIME(2);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::kTmemCols);
   }
-  if (PARTIALS) return;
+  FLEXQ_CTA_TIME(5);
+  if (PARTIALS) {
+    FLEXQ_CTA_TIME(3);
+    return;
+  }
 
   const bool is_epi = warp >= 6;
   const int e = warp - 6;
@@ -450,6 +507,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     // split-K: ranks 1..S-1 add their partial tiles into rank 0's shared
     // memory (the stage ring is idle now), in a fixed order
     cluster_sync_all();
+    FLEXQ_CTA_TIME(6);
     if (is_epi && ks != 0) {
       const uint32_t remote = map_to_rank(smem_u32(red), 0);
 #pragma unroll
@@ -459,7 +517,10 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       }
     }
     cluster_sync_all();
-    if (ks != 0) return;
+    if (ks != 0) {
+      FLEXQ_CTA_TIME(3);
+      return;
+    }
     if (is_epi) {
       for (int r = 1; r < S; ++r) {
 #pragma unroll
@@ -468,6 +529,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       }
     }
   }
+  FLEXQ_CTA_TIME(7);
   if (is_epi) {
     const int n = nt * kTileRows + row;
 #pragma unroll
@@ -476,6 +538,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       if (m < M) args.y[static_cast<size_t>(m) * N + n] = __float2half_rn(acc[j]);
     }
   }
+  FLEXQ_CTA_TIME(3);
 }
 
 }  // namespace flexq

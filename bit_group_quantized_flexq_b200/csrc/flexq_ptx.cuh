@@ -41,15 +41,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar,
                : "memory");
 }
 
+// One probe of the phase; the hardware may suspend the calling thread for up
+// to `suspend_ns` while the phase is still incomplete (it wakes on completion).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr,
-                                              uint32_t parity) {
+                                              uint32_t parity,
+                                              uint32_t suspend_ns = 1000000u) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
-      : "r"(bar_addr), "r"(parity)
+      : "r"(bar_addr), "r"(parity), "r"(suspend_ns)
       : "memory");
   return done != 0;
 }
