@@ -456,23 +456,24 @@ int flexq_get_device_status(void* stream) {
   if (h[0] == 0) return ok();
   e = cudaMemset(st->status, 0, sizeof(h));
   if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
-  static const char* roles[] = {"producer", "mma", "unpack(full)", "unpack(a_empty)", "epilogue"};
+  static const char* roles[] = {"producer", "mma", "unpack", "?", "epilogue (partials)",
+                                "epilogue (scales)"};
   return fail(static_cast<int>(h[0]), "device wait timed out in the %s role of block %u",
-              h[1] < 5 ? roles[h[1]] : "?", h[2]);
+              h[1] < 6 ? roles[h[1]] : "?", h[2]);
 }
 
 #ifdef FLEXQ_TRACE
-// Trace builds only: copies the pipeline trace of the last GEMM launch.
-int flexq_debug_read_trace(long long* host, size_t count) {
+// Trace builds only: per-role loop/wait cycles of CTA 0 and of the middle CTA
+// ([2][4][4]) and the per-CTA timeline ([8192][8]) of the last launch.
+int flexq_debug_read_roles(long long* host, size_t count) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-  const size_t n = sizeof(flexq::g_flexq_trace) / sizeof(long long);
-  e = cudaMemcpyFromSymbol(host, flexq::g_flexq_trace, (count < n ? count : n) * sizeof(long long));
-  if (e != cudaSuccess) return cuda_fail(e, "reading the trace");
+  const size_t n = sizeof(flexq::g_flexq_role) / sizeof(long long);
+  e = cudaMemcpyFromSymbol(host, flexq::g_flexq_role, (count < n ? count : n) * sizeof(long long));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the role trace");
   return ok();
 }
 
-// Trace builds only: copies the per-CTA timeline ([cta][8]) of the last launch.
 int flexq_debug_read_cta_times(unsigned long long* host, size_t count) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");

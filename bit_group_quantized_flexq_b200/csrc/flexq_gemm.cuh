@@ -20,11 +20,11 @@
 //               (12288 B) per 128-wide K block into a STAGES-deep ring;
 //   warp 1      TMEM allocator and MMA issuer: 4 MMAs (K = 32 each) per K
 //               block into the int32 partial buffer of the current group
-//               (double buffered, T columns each), commits per group;
+//               (kPBufs buffers of T columns), commits per group;
 //   warps 2..5  unpack: each thread owns one weight row, turns its 96 packed
 //               bytes into 128 int8 codes (code * 4, the 6-bit field in the
-//               top of each byte) and stores them into a TMEM A slot (4
-//               slots of 32 columns);
+//               top of each byte) and stores them into the TMEM A slot of
+//               the stage (32 columns per stage);
 //   warps 6..   epilogue: per group, load the int32 partials from TMEM,
 //               release the buffer, and accumulate
 //               acc += float(P) * (sw[n,g]/4 * sa[m,g]) in FP32 registers;
@@ -42,7 +42,6 @@ namespace flexq {
 constexpr int kTileRows = 128;        // weight rows per tile (MMA M)
 constexpr int kKBlock = 128;          // codes per K block
 constexpr int kWTileBytes = 12288;    // packed bytes of a 128 x 128 tile
-constexpr int kASlots = 4;            // TMEM A ring depth
 constexpr int kStatusTimeout = 5;     // == FLEXQ_ERR_DEVICE_TIMEOUT
 
 struct GemmArgs {
@@ -73,9 +72,17 @@ struct GemmCfg {
   static constexpr int kScSaBytes = 8 * T * 2;
   static constexpr int kScSlotBytes = kScSaBytes + 8 * 128 * 2;
   static constexpr int kMainBytes = kStages * kStageBytes + kScSlots * kScSlotBytes;
+  // int32 partial buffers in TMEM (one per group in flight), then the A ring
+  // TMEM: int32 partial buffers (one per group in flight), then one A slot
+  // (32 columns = 128 int8 codes per row) per shared-memory stage.  A slot s
+  // is only rewritten for K block i after the producer refilled stage s for
+  // i, which it does only after the MMAs of K block i - STAGES (the previous
+  // user of slot s) have completed, so the slot needs no barrier of its own.
+  static constexpr int kPBufs = (T == 16) ? 4 : (T == 32) ? 3 : (T == 64) ? 2 : 3;
   static constexpr int kPCol0 = 0;
-  static constexpr int kACol0 = 2 * T;
-  static constexpr int kTmemCols = (2 * T + 128 <= 256) ? 256 : 512;
+  static constexpr int kACol0 = kPBufs * T;
+  static constexpr int kTmemCols = (kACol0 + 32 * kStages <= 256) ? 256 : 512;
+  static_assert(kACol0 + 32 * kStages <= kTmemCols, "TMEM budget");
   static constexpr int kLdChunk = (T == 128) ? 32 : 16;   // TMEM columns per load batch
   static_assert(kCols % 16 == 0, "epilogue column chunking");
 };
@@ -84,10 +91,9 @@ template <int T>
 struct GemmCtrl {
   uint64_t full[GemmCfg<T>::kStages];
   uint64_t empty[GemmCfg<T>::kStages];
-  uint64_t a_full[kASlots];
-  uint64_t a_empty[kASlots];
-  uint64_t p_full[2];
-  uint64_t p_empty[2];
+  uint64_t a_full[GemmCfg<T>::kStages];
+  uint64_t p_full[GemmCfg<T>::kPBufs];
+  uint64_t p_empty[GemmCfg<T>::kPBufs];
   uint64_t s_full[GemmCfg<T>::kScSlots];
   uint64_t s_empty[GemmCfg<T>::kScSlots];
   uint64_t done;
@@ -97,19 +103,17 @@ struct GemmCtrl {
   float sa[GemmCfg<T>::kEpiWarps][8][GemmCfg<T>::kCols];
 };
 
-// Optional pipeline trace (compile with -DFLEXQ_TRACE): CTA (0,0,0) records
-// clock64() offsets at fixed points of each role, [role][event][index], and
-// every CTA records %globaltimer at entry (0), after set-up (1), after its
-// roles' loops (2), at exit (3), after the TMEM release (5), after the first
-// cluster barrier (6) and before the output store (7); its SM id in slot 4.
+// Optional pipeline trace (compile with -DFLEXQ_TRACE).  Every CTA records
+// %globaltimer at entry (0), after set-up (1), after its roles' loops (2), at
+// exit (3), after the TMEM release (5), after the first cluster barrier (6)
+// and before the output store (7), with its SM id in slot 4.  CTA 0 and the
+// CTA in the middle of the grid also record, per role (producer, MMA, unpack
+// warp of lane quarter 0, first epilogue warp), the cycles spent in the role
+// loop, the cycles spent waiting on barriers and the iteration count:
+// g_flexq_role[which CTA][role][0..2].
 #ifdef FLEXQ_TRACE
-__device__ long long g_flexq_trace[4][4][1024];
 __device__ unsigned long long g_flexq_cta_times[8192][8];
-#define FLEXQ_TRACE_POINT(role, ev, idx, t0)                                   \
-  do {                                                                         \
-    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (idx) < 1024) \
-      g_flexq_trace[role][ev][idx] = clock64() - (t0);                         \
-  } while (0)
+__device__ long long g_flexq_role[2][4][4];
 #define FLEXQ_CTA_TIME(slot)                                                   \
   do {                                                                         \
     const unsigned cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
@@ -120,12 +124,33 @@ __device__ unsigned long long g_flexq_cta_times[8192][8];
       g_flexq_cta_times[cta_][4] = smid_;                                      \
     }                                                                          \
   } while (0)
-#else
-#define FLEXQ_TRACE_POINT(role, ev, idx, t0) \
-  do {                                       \
+#define FLEXQ_ROLE_CLOCK long long fx_wait_ = 0, fx_t0_ = clock64()
+#define FLEXQ_WAIT(expr)                       \
+  ({                                           \
+    const long long fx_w0_ = clock64();        \
+    const bool fx_r_ = (expr);                 \
+    fx_wait_ += clock64() - fx_w0_;            \
+    fx_r_;                                     \
+  })
+#define FLEXQ_ROLE_DONE(role, iters)                                             \
+  do {                                                                           \
+    const unsigned cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
+    const unsigned mid_ = (gridDim.x * gridDim.y * gridDim.z) / 2;              \
+    if (cta_ == 0 || cta_ == mid_) {                                             \
+      const int w_ = cta_ == 0 ? 0 : 1;                                          \
+      g_flexq_role[w_][role][0] = clock64() - fx_t0_;                            \
+      g_flexq_role[w_][role][1] = fx_wait_;                                      \
+      g_flexq_role[w_][role][2] = (iters);                                       \
+    }                                                                            \
   } while (0)
+#else
 #define FLEXQ_CTA_TIME(slot) \
   do {                       \
+  } while (0)
+#define FLEXQ_ROLE_CLOCK
+#define FLEXQ_WAIT(expr) (expr)
+#define FLEXQ_ROLE_DONE(role, iters) \
+  do {                               \
   } while (0)
 #endif
 
@@ -211,19 +236,19 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   const int u1 = static_cast<int>((static_cast<long long>(ks + 1) * units) / S);
   const int kb0 = u0 * U;
   const int nkb = (u1 - u0) * U;
-  const int g0 = kb0 * kKBlock / gs;
-  const int ngroups = nkb * kKBlock / gs;
+  // gs is a power of two (32..256): group arithmetic uses masks and shifts
+  const int gs_log2 = __ffs(gs) - 1;
+  const int gs_mask = gs - 1;
+  const int g0 = (kb0 * kKBlock) >> gs_log2;
+  const int ngroups = (nkb * kKBlock) >> gs_log2;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&ctrl->full[s], 1);
       mbar_init(&ctrl->empty[s], 4 + 1);     // 4 unpack warps + MMA commit
     }
-    for (int s = 0; s < kASlots; ++s) {
-      mbar_init(&ctrl->a_full[s], 4);
-      mbar_init(&ctrl->a_empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
+    for (int s = 0; s < STAGES; ++s) mbar_init(&ctrl->a_full[s], 4);
+    for (int b = 0; b < Cfg::kPBufs; ++b) {
       mbar_init(&ctrl->p_full[b], 1);
       mbar_init(&ctrl->p_empty[b], Cfg::kEpiWarps);
     }
@@ -244,8 +269,6 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
-  const long long t_start = clock64();
-  (void)t_start;
   FLEXQ_CTA_TIME(1);
 
   // epilogue state lives across the role switch below
@@ -256,17 +279,18 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   if (warp == 0) {
     // ------------------------------------------------------- producer ----
     if (lane == 0) {
+      FLEXQ_ROLE_CLOCK;
       uint32_t issued = 0, parity = 0, sc_issued = 0, sc_parity = 0;
       const int n_oct = PARTIALS ? 0 : (ngroups + 7) / 8;
       int next_oct = 0;
       bool ok = true;
       for (int i = 0; i < nkb && ok; ++i) {
         // scales: issue octet o at the first K block that touches group 8*o
-        const int lg_first = i * kKBlock / gs;
+        const int lg_first = (i * kKBlock) >> gs_log2;
         while (next_oct < n_oct && next_oct * 8 <= lg_first) {
           const int o = next_oct, slot = o % Cfg::kScSlots;
           if (o >= Cfg::kScSlots &&
-              !mbar_wait(&ctrl->s_empty[slot], ((o / Cfg::kScSlots) - 1) & 1, lim)) {
+              !FLEXQ_WAIT(mbar_wait(&ctrl->s_empty[slot], ((o / Cfg::kScSlots) - 1) & 1, lim))) {
             ok = false;
             break;
           }
@@ -283,7 +307,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         if (!ok) break;
         const int s = i % STAGES;
         if (i >= STAGES &&
-            !mbar_wait(&ctrl->empty[s], ((i / STAGES) - 1) & 1, lim)) {
+            !FLEXQ_WAIT(mbar_wait(&ctrl->empty[s], ((i / STAGES) - 1) & 1, lim))) {
           ok = false;
           break;
         }
@@ -296,9 +320,9 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
                   kWTileBytes, &ctrl->full[s]);
         issued |= 1u << s;
         parity = (parity & ~(1u << s)) | (static_cast<uint32_t>((i / STAGES) & 1) << s);
-        FLEXQ_TRACE_POINT(0, 0, i, t_start);
       }
       if (!ok) record_status(args.status, kStatusTimeout, 0);
+      FLEXQ_ROLE_DONE(0, nkb);
       // every issued copy must land before the CTA may finish
       for (int s = 0; s < STAGES; ++s)
         if ((issued >> s) & 1u) mbar_wait(&ctrl->full[s], (parity >> s) & 1u, lim);
@@ -308,50 +332,57 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     __syncwarp();
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA -----
+    // Running counters instead of divisions: stage s / phase, accumulator
+    // buffer b / pass, and the position of the next 32-wide MMA in its group.
     if (lane == 0) {
+      FLEXQ_ROLE_CLOCK;
       constexpr uint32_t idesc = idesc_i8(kTileRows, T);
-      int lg = 0;
+      const uint32_t mmas_per_group_mask = static_cast<uint32_t>(gs >> 5) - 1u;
+      const uint64_t desc0 = smem_desc_k_sw128(smem_u32(xs_ring));
+      const uint32_t a_col0 = tmem + Cfg::kACol0;
+      uint32_t s = 0, phase = 0, b = 0, gsub = 0;
+      int pass = 0;
       bool ok = true;
       for (int i = 0; i < nkb && ok; ++i) {
-        const int s = i % STAGES;
-        const int slot = i & (kASlots - 1);
-        if (!mbar_wait(&ctrl->full[s], (i / STAGES) & 1, lim) ||
-            !mbar_wait(&ctrl->a_full[slot], (i / kASlots) & 1, lim)) {
+        if (!FLEXQ_WAIT(mbar_wait(&ctrl->full[s], phase, lim)) ||
+            !FLEXQ_WAIT(mbar_wait(&ctrl->a_full[s], phase, lim))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        FLEXQ_TRACE_POINT(1, 0, i, t_start);
-        const uint32_t xs_addr = smem_u32(xs_ring + s * Cfg::kXsBytes);
+        // the start-address field of the descriptor is addr >> 4 in its low
+        // 14 bits; shared addresses stay below 2^18, so plain adds are exact
+        const uint64_t desc = desc0 + ((s * Cfg::kXsBytes) >> 4);
+        const uint32_t a_col = a_col0 + s * 32;
 #pragma unroll
         for (int sub = 0; sub < 4; ++sub) {
-          const int kk = (kb0 + i) * kKBlock + sub * 32;
-          const bool first = (kk % gs) == 0;
-          const bool last = ((kk + 32) % gs) == 0;
-          const int b = lg & 1;
-          if (first && lg >= 2) {
-            if (!mbar_wait(&ctrl->p_empty[b], ((lg >> 1) - 1) & 1, lim)) {
+          if (gsub == 0 && pass > 0) {
+            if (!FLEXQ_WAIT(mbar_wait(&ctrl->p_empty[b], (pass - 1) & 1, lim))) {
               ok = false;
               break;
             }
             tc_fence_after();
           }
-          if (first) FLEXQ_TRACE_POINT(1, 1, lg, t_start);
-          mma_i8_tmem_a(tmem + Cfg::kPCol0 + b * T,
-                        tmem + Cfg::kACol0 + slot * 32 + sub * 8,
-                        smem_desc_k_sw128(xs_addr + sub * 32), idesc,
-                        first ? 0u : 1u);
-          if (last) {
+          mma_i8_tmem_a(tmem + Cfg::kPCol0 + b * T, a_col + sub * 8, desc + (sub * 32 >> 4),
+                        idesc, gsub != 0 ? 1u : 0u);
+          if (gsub == mmas_per_group_mask) {
             mma_commit(&ctrl->p_full[b]);
-            ++lg;
+            if (++b == Cfg::kPBufs) {
+              b = 0;
+              ++pass;
+            }
           }
+          gsub = (gsub + 1) & mmas_per_group_mask;
         }
         if (!ok) break;
-        mma_commit(&ctrl->empty[s]);
-        mma_commit(&ctrl->a_empty[slot]);
-        FLEXQ_TRACE_POINT(1, 2, i, t_start);
+        mma_commit(&ctrl->empty[s]);       // frees smem stage s and A slot s
+        if (++s == STAGES) {
+          s = 0;
+          phase ^= 1;
+        }
       }
       if (!ok) record_status(args.status, kStatusTimeout, 1);
+      FLEXQ_ROLE_DONE(1, nkb);
       // all issued MMAs must finish before TMEM is released
       mma_commit(&ctrl->done);
       mbar_wait(&ctrl->done, 0, lim);
@@ -362,13 +393,13 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     const int q = warp & 3;                       // TMEM lane quarter
     const int row = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    FLEXQ_ROLE_CLOCK;
     for (int i = 0; i < nkb; ++i) {
       const int s = i % STAGES;
-      if (!warp_wait(&ctrl->full[s], (i / STAGES) & 1, lim)) {
+      if (!FLEXQ_WAIT(warp_wait(&ctrl->full[s], (i / STAGES) & 1, lim))) {
         if (lane == 0) record_status(args.status, kStatusTimeout, 2);
         break;
       }
-      if (q == 0 && lane == 0) FLEXQ_TRACE_POINT(2, 0, i, t_start);
       const uint4* src = reinterpret_cast<const uint4*>(w_ring + s * kWTileBytes) + row;
       uint32_t wa[12], wb[12];
 #pragma unroll
@@ -380,14 +411,8 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->empty[s]);
-      const int slot = i & (kASlots - 1);
-      if (i >= kASlots &&
-          !warp_wait(&ctrl->a_empty[slot], ((i / kASlots) - 1) & 1, lim)) {
-        if (lane == 0) record_status(args.status, kStatusTimeout, 3);
-        break;
-      }
+      const int slot = s;                   // free: see GemmCfg
       tc_fence_after();
-      if (q == 0 && lane == 0) FLEXQ_TRACE_POINT(2, 1, i, t_start);
       const uint32_t col = tmem + lane_base + Cfg::kACol0 + slot * 32;
       uint32_t out[16];
       unpack48(wa, out);
@@ -398,8 +423,8 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->a_full[slot]);
-      if (q == 0 && lane == 0) FLEXQ_TRACE_POINT(2, 2, i, t_start);
     }
+    if (q == 0 && lane == 0) FLEXQ_ROLE_DONE(2, nkb);
   } else {
     // ------------------------------------------------------ epilogue -----
     const int e = warp - 6;
@@ -410,8 +435,9 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     const int col0 = c * Cfg::kCols;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const int m_base = mt * T + col0;
+    FLEXQ_ROLE_CLOCK;
     for (int lg = 0; lg < ngroups; ++lg) {
-      const int b = lg & 1;
+      const int b = lg % Cfg::kPBufs;
       const int g = g0 + lg;
       const int gi = lg & 7;
       const int sc_slot = (lg >> 3) % Cfg::kScSlots;
@@ -419,11 +445,10 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       float swn = 0.0f;
       if (!PARTIALS) {
         if (gi == 0) {
-          if (!warp_wait(&ctrl->s_full[sc_slot], ((lg >> 3) / Cfg::kScSlots) & 1, lim)) {
+          if (!FLEXQ_WAIT(warp_wait(&ctrl->s_full[sc_slot], ((lg >> 3) / Cfg::kScSlots) & 1, lim))) {
             if (lane == 0) record_status(args.status, kStatusTimeout, 5);
             break;
           }
-          if (e == 0 && lane == 0) FLEXQ_TRACE_POINT(3, 0, lg >> 3, t_start);
           // this warp's tokens of the octet, FP16 -> FP32, into its own buffer
           const __half* sa_h = reinterpret_cast<const __half*>(sc);
           __syncwarp();
@@ -438,12 +463,11 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         swn = __half2float(sw_h[gi * kTileRows + row]) * 0.25f;   // TMEM holds 4 * code
       }
       const float* sa_w = ctrl->sa[e][gi];
-      if (!warp_wait(&ctrl->p_full[b], (lg >> 1) & 1, lim)) {
+      if (!FLEXQ_WAIT(warp_wait(&ctrl->p_full[b], (lg / Cfg::kPBufs) & 1, lim))) {
         if (lane == 0) record_status(args.status, kStatusTimeout, 4);
         break;
       }
       tc_fence_after();
-      if (e == 0 && lane == 0) FLEXQ_TRACE_POINT(3, 1, lg, t_start);
       // drain the partials in chunks; the buffer is released right after the
       // last chunk has been read, before that chunk's arithmetic
       constexpr int CH = Cfg::kLdChunk;
@@ -460,7 +484,6 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctrl->p_empty[b]);
-          if (e == 0 && lane == 0) FLEXQ_TRACE_POINT(3, 2, lg, t_start);
         }
         if (PARTIALS) {
 #pragma unroll
@@ -477,12 +500,12 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
                                     swn * sa_w[ch * CH + j], acc[ch * CH + j]);
         }
       }
-      if (e == 0 && lane == 0) FLEXQ_TRACE_POINT(3, 3, lg, t_start);
       if (!PARTIALS && (gi == 7 || lg == ngroups - 1)) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->s_empty[sc_slot]);
       }
     }
+    if (e == 0 && lane == 0) FLEXQ_ROLE_DONE(3, ngroups);
   }
 
   // ------------------------------------------------------------ teardown --

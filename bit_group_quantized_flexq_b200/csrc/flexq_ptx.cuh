@@ -57,11 +57,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr,
   return done != 0;
 }
 
+// Non-blocking probe of the phase.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar_addr, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 // Waits until the phase with the given parity has completed.  Gives up after
 // `limit_ns` nanoseconds and returns false; never spins without bound.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
+  if (mbar_test_wait(a, parity)) return true;
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
