@@ -100,7 +100,7 @@ struct GemmCtrl {
   uint32_t tmem_base;
   uint32_t pad;
   // per epilogue warp: its tokens' activation scales of the current octet, FP32
-  float sa[GemmCfg<T>::kEpiWarps][8][GemmCfg<T>::kCols];
+  alignas(16) float sa[GemmCfg<T>::kEpiWarps][8][GemmCfg<T>::kCols];
 };
 
 // Optional pipeline trace (compile with -DFLEXQ_TRACE).  Every CTA records
@@ -238,7 +238,6 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   const int nkb = (u1 - u0) * U;
   // gs is a power of two (32..256): group arithmetic uses masks and shifts
   const int gs_log2 = __ffs(gs) - 1;
-  const int gs_mask = gs - 1;
   const int g0 = (kb0 * kKBlock) >> gs_log2;
   const int ngroups = (nkb * kKBlock) >> gs_log2;
 
@@ -272,9 +271,10 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   FLEXQ_CTA_TIME(1);
 
   // epilogue state lives across the role switch below
-  float acc[Cfg::kCols];
+  // FP32 accumulators as pairs (packed f32x2 arithmetic: sm_100 FFMA2/FMUL2)
+  float2 acc[Cfg::kCols / 2];
 #pragma unroll
-  for (int j = 0; j < Cfg::kCols; ++j) acc[j] = 0.0f;
+  for (int j = 0; j < Cfg::kCols / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
 
   if (warp == 0) {
     // ------------------------------------------------------- producer ----
@@ -332,54 +332,67 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     __syncwarp();
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA -----
-    // Running counters instead of divisions: stage s / phase, accumulator
-    // buffer b / pass, and the position of the next 32-wide MMA in its group.
+    // The issuing thread shares its SM sub-partition with busy unpack and
+    // epilogue warps, so every instruction on its path counts: the loop is
+    // unrolled over the stages (addresses become constants) and the group
+    // boundaries of the four 32-wide MMAs of a K block come from two 4-bit
+    // masks (indexed by the K block's parity, which matters for gs = 256).
     if (lane == 0) {
       FLEXQ_ROLE_CLOCK;
       constexpr uint32_t idesc = idesc_i8(kTileRows, T);
-      const uint32_t mmas_per_group_mask = static_cast<uint32_t>(gs >> 5) - 1u;
-      const uint64_t desc0 = smem_desc_k_sw128(smem_u32(xs_ring));
-      const uint32_t a_col0 = tmem + Cfg::kACol0;
-      uint32_t s = 0, phase = 0, b = 0, gsub = 0;
-      int pass = 0;
-      bool ok = true;
-      for (int i = 0; i < nkb && ok; ++i) {
-        if (!FLEXQ_WAIT(mbar_wait(&ctrl->full[s], phase, lim)) ||
-            !FLEXQ_WAIT(mbar_wait(&ctrl->a_full[s], phase, lim))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // the start-address field of the descriptor is addr >> 4 in its low
-        // 14 bits; shared addresses stay below 2^18, so plain adds are exact
-        const uint64_t desc = desc0 + ((s * Cfg::kXsBytes) >> 4);
-        const uint32_t a_col = a_col0 + s * 32;
+      uint32_t first_mask[2], last_mask[2];
+#pragma unroll
+      for (int par = 0; par < 2; ++par) {
+        first_mask[par] = last_mask[par] = 0;
 #pragma unroll
         for (int sub = 0; sub < 4; ++sub) {
-          if (gsub == 0 && pass > 0) {
-            if (!FLEXQ_WAIT(mbar_wait(&ctrl->p_empty[b], (pass - 1) & 1, lim))) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-          }
-          mma_i8_tmem_a(tmem + Cfg::kPCol0 + b * T, a_col + sub * 8, desc + (sub * 32 >> 4),
-                        idesc, gsub != 0 ? 1u : 0u);
-          if (gsub == mmas_per_group_mask) {
-            mma_commit(&ctrl->p_full[b]);
-            if (++b == Cfg::kPBufs) {
-              b = 0;
-              ++pass;
-            }
-          }
-          gsub = (gsub + 1) & mmas_per_group_mask;
+          const int kk = par * kKBlock + sub * 32;    // K-block ranges start group-aligned
+          if ((kk & (gs - 1)) == 0) first_mask[par] |= 1u << sub;
+          if (((kk + 32) & (gs - 1)) == 0) last_mask[par] |= 1u << sub;
         }
-        if (!ok) break;
-        mma_commit(&ctrl->empty[s]);       // frees smem stage s and A slot s
-        if (++s == STAGES) {
-          s = 0;
-          phase ^= 1;
+      }
+      const uint64_t desc0 = smem_desc_k_sw128(smem_u32(xs_ring));
+      const uint32_t a_col0 = tmem + Cfg::kACol0;
+      uint32_t phase = 0, b = 0;
+      int pass = 0;
+      bool ok = true;
+      for (int i0 = 0; i0 < nkb && ok; i0 += STAGES) {
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) {
+          const int i = i0 + s;
+          if (i >= nkb) break;
+          if (!FLEXQ_WAIT(mbar_wait(&ctrl->full[s], phase, lim)) ||
+              !FLEXQ_WAIT(mbar_wait(&ctrl->a_full[s], phase, lim))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t fm = first_mask[i & 1], lm = last_mask[i & 1];
+#pragma unroll
+          for (int sub = 0; sub < 4; ++sub) {
+            const bool first = (fm >> sub) & 1u;
+            if (first && pass > 0) {
+              if (!FLEXQ_WAIT(mbar_wait(&ctrl->p_empty[b], (pass - 1) & 1, lim))) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            mma_i8_tmem_a(tmem + Cfg::kPCol0 + b * T, a_col0 + s * 32 + sub * 8,
+                          desc0 + ((s * Cfg::kXsBytes + sub * 32) >> 4), idesc,
+                          first ? 0u : 1u);
+            if ((lm >> sub) & 1u) {
+              mma_commit(&ctrl->p_full[b]);
+              if (++b == Cfg::kPBufs) {
+                b = 0;
+                ++pass;
+              }
+            }
+          }
+          if (!ok) break;
+          mma_commit(&ctrl->empty[s]);     // frees smem stage s and A slot s
         }
+        phase ^= 1;
       }
       if (!ok) record_status(args.status, kStatusTimeout, 1);
       FLEXQ_ROLE_DONE(1, nkb);
@@ -494,10 +507,22 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
                   static_cast<int32_t>(pv[j]) >> 2;
           }
         } else {
+          // acc += float(P) * (sw/4 * sa), two columns per instruction; the
+          // FP16 x FP16 scale product is exact in FP32, the FMA rounds once
+          const float2 swn2 = make_float2(swn, swn);
+          const float4* sa4 = reinterpret_cast<const float4*>(sa_w + ch * CH);
 #pragma unroll
-          for (int j = 0; j < CH; ++j)
-            acc[ch * CH + j] = fmaf(static_cast<float>(static_cast<int32_t>(pv[j])),
-                                    swn * sa_w[ch * CH + j], acc[ch * CH + j]);
+          for (int j = 0; j < CH; j += 4) {
+            const float4 s4 = sa4[j / 4];
+            const float2 s_lo = __fmul2_rn(swn2, make_float2(s4.x, s4.y));
+            const float2 s_hi = __fmul2_rn(swn2, make_float2(s4.z, s4.w));
+            const float2 p_lo = make_float2(__int2float_rn(static_cast<int32_t>(pv[j])),
+                                            __int2float_rn(static_cast<int32_t>(pv[j + 1])));
+            const float2 p_hi = make_float2(__int2float_rn(static_cast<int32_t>(pv[j + 2])),
+                                            __int2float_rn(static_cast<int32_t>(pv[j + 3])));
+            acc[(ch * CH + j) / 2] = __ffma2_rn(p_lo, s_lo, acc[(ch * CH + j) / 2]);
+            acc[(ch * CH + j) / 2 + 1] = __ffma2_rn(p_hi, s_hi, acc[(ch * CH + j) / 2 + 1]);
+          }
         }
       }
       if (!PARTIALS && (gi == 7 || lg == ngroups - 1)) {
@@ -536,7 +561,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
 #pragma unroll
       for (int j = 0; j < Cfg::kCols; ++j) {
         const uint32_t off = static_cast<uint32_t>(((ks - 1) * T + col0 + j) * kTileRows + row);
-        st_cluster_f32(remote + off * 4u, acc[j]);
+        st_cluster_f32(remote + off * 4u, (j & 1) ? acc[j / 2].y : acc[j / 2].x);
       }
     }
     cluster_sync_all();
@@ -547,8 +572,10 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     if (is_epi) {
       for (int r = 1; r < S; ++r) {
 #pragma unroll
-        for (int j = 0; j < Cfg::kCols; ++j)
-          acc[j] += red[((r - 1) * T + col0 + j) * kTileRows + row];
+        for (int j = 0; j < Cfg::kCols; j += 2) {
+          acc[j / 2].x += red[((r - 1) * T + col0 + j) * kTileRows + row];
+          acc[j / 2].y += red[((r - 1) * T + col0 + j + 1) * kTileRows + row];
+        }
       }
     }
   }
@@ -558,7 +585,9 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
 #pragma unroll
     for (int j = 0; j < Cfg::kCols; ++j) {
       const int m = mt * T + col0 + j;
-      if (m < M) args.y[static_cast<size_t>(m) * N + n] = __float2half_rn(acc[j]);
+      if (m < M)
+        args.y[static_cast<size_t>(m) * N + n] =
+            __float2half_rn((j & 1) ? acc[j / 2].y : acc[j / 2].x);
     }
   }
   FLEXQ_CTA_TIME(3);
