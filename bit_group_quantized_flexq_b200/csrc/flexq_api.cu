@@ -109,7 +109,7 @@ int check_gemm_shape(int M, int N, int K, int gs) {
     return fail(FLEXQ_ERR_INVALID_ARG, "sizes must be M >= 0, N > 0, K > 0 (M=%d N=%d K=%d)", M, N, K);
   if (!valid_gs(gs)) return fail(FLEXQ_ERR_UNSUPPORTED, "group_size %d not in {32,64,128,256}", gs);
   if (N % 128) return fail(FLEXQ_ERR_UNSUPPORTED, "N=%d is not a multiple of 128", N);
-  if (K % 128) return fail(FLEXQ_ERR_UNSUPPORTED, "K=%d is not a multiple of 128", K);
+  if (K % 256) return fail(FLEXQ_ERR_UNSUPPORTED, "K=%d is not a multiple of 256", K);
   if (K % gs) return fail(FLEXQ_ERR_UNSUPPORTED, "K=%d is not a multiple of group_size %d", K, gs);
   if (N / 128 > 65535) return fail(FLEXQ_ERR_UNSUPPORTED, "N=%d too large", N);
   return FLEXQ_OK;
@@ -141,7 +141,7 @@ struct Plan {
 
 Plan make_plan(int M, int N, int K, int gs, int sms, bool partials) {
   Plan p;
-  const int units = (K / 128) / (gs > 128 ? gs / 128 : 1);
+  const int units = K / 256;                          // K stages of the kernel
   p.T = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
   const long long tiles = static_cast<long long>(N / 128) * ((M + p.T - 1) / p.T);
   const long long slots = static_cast<long long>(sms) * (p.T <= 64 ? 2 : 1);
@@ -326,7 +326,7 @@ const char* flexq_last_error_message(void) { return t_last_error.c_str(); }
 size_t flexq_act_scales_ld(int M) { return M > 0 ? static_cast<size_t>(act_scales_ld(M)) : 0; }
 
 size_t flexq_weight_packed_bytes(int N, int K, int group_size) {
-  if (N <= 0 || K <= 0 || N % 128 || K % 128 || !valid_gs(group_size) || K % group_size) return 0;
+  if (N <= 0 || K <= 0 || N % 128 || K % 256 || !valid_gs(group_size) || K % group_size) return 0;
   return static_cast<size_t>(N) * static_cast<size_t>(K) / 4 * 3;
 }
 

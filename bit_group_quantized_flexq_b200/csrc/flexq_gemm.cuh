@@ -14,17 +14,22 @@
 // contiguous, group-aligned range of K (a cluster of `split` CTAs shares the
 // output tile and reduces through distributed shared memory).
 //
+// The pipeline advances in stages of 256 codes of K (two 128 x 128 weight
+// tiles), which halves the barrier traffic per byte against one tile per
+// stage.
+//
 // Warp roles (all pipeline waits are bounded, see mbar_wait):
-//   warp 0      producer: TMA tile of the int8 activations (T rows x 128 B,
-//               128-byte swizzle) + bulk copy of the packed weight tile
-//               (12288 B) per 128-wide K block into a STAGES-deep ring;
-//   warp 1      TMEM allocator and MMA issuer: 4 MMAs (K = 32 each) per K
-//               block into the int32 partial buffer of the current group
+//   warp 0      producer: per stage, two TMA boxes of the int8 activations
+//               (T rows x 128 B each, 128-byte swizzle) and one 24576-byte
+//               bulk copy of two consecutive packed weight tiles into a
+//               STAGES-deep ring; per 8 groups, the group scales;
+//   warp 1      TMEM allocator and MMA issuer: 8 MMAs (K = 32 each) per
+//               stage into the int32 partial buffer of the current group
 //               (kPBufs buffers of T columns), commits per group;
-//   warps 2..5  unpack: each thread owns one weight row, turns its 96 packed
-//               bytes into 128 int8 codes (code * 4, the 6-bit field in the
+//   warps 2..5  unpack: each thread owns one weight row, turns its 192 packed
+//               bytes into 256 int8 codes (code * 4, the 6-bit field in the
 //               top of each byte) and stores them into the TMEM A slot of
-//               the stage (32 columns per stage);
+//               the stage (64 columns per stage);
 //   warps 6..   epilogue: per group, load the int32 partials from TMEM,
 //               release the buffer, and accumulate
 //               acc += float(P) * (sw[n,g]/4 * sa[m,g]) in FP32 registers;
@@ -60,11 +65,14 @@ struct GemmCfg {
   static constexpr int kEpiWarps = (T <= 32) ? 4 : 8;
   static constexpr int kThreads = (6 + kEpiWarps) * 32;
   static constexpr int kCols = T / (kEpiWarps / 4);      // tokens per epi warp
-  static constexpr int kStages = (T == 16) ? 6 : (T == 32) ? 5 : 4;
+  static constexpr int kStages = (T == 64) ? 2 : 3;
   static constexpr int kMinBlocks = (T <= 64) ? 2 : 1;
   static constexpr int kMaxSplit = (T == 16) ? 8 : (T == 32) ? 6 : (T == 64) ? 4 : 2;
-  static constexpr int kXsBytes = T * 128;
-  static constexpr int kStageBytes = kXsBytes + kWTileBytes;
+  static constexpr int kKStage = 2 * kKBlock;            // codes of K per stage
+  static constexpr int kXsHalf = T * 128;                // one activation box
+  static constexpr int kXsBytes = 2 * kXsHalf;
+  static constexpr int kWStageBytes = 2 * kWTileBytes;
+  static constexpr int kStageBytes = kXsBytes + kWStageBytes;
   // scale ring: one slot holds 8 groups ("octet") of activation scales for
   // the T tokens ([8][T] fp16) and of weight scales for the 128 rows
   // ([8][128] fp16), each brought by one TMA box
@@ -72,17 +80,17 @@ struct GemmCfg {
   static constexpr int kScSaBytes = 8 * T * 2;
   static constexpr int kScSlotBytes = kScSaBytes + 8 * 128 * 2;
   static constexpr int kMainBytes = kStages * kStageBytes + kScSlots * kScSlotBytes;
-  // int32 partial buffers in TMEM (one per group in flight), then the A ring
   // TMEM: int32 partial buffers (one per group in flight), then one A slot
-  // (32 columns = 128 int8 codes per row) per shared-memory stage.  A slot s
-  // is only rewritten for K block i after the producer refilled stage s for
-  // i, which it does only after the MMAs of K block i - STAGES (the previous
+  // (64 columns = 256 int8 codes per row) per shared-memory stage.  A slot s
+  // is only rewritten for stage i after the producer refilled stage s for
+  // i, which it does only after the MMAs of stage i - STAGES (the previous
   // user of slot s) have completed, so the slot needs no barrier of its own.
-  static constexpr int kPBufs = (T == 16) ? 4 : (T == 32) ? 3 : (T == 64) ? 2 : 3;
+  static constexpr int kPBufs = (T == 16) ? 4 : 2;
   static constexpr int kPCol0 = 0;
   static constexpr int kACol0 = kPBufs * T;
-  static constexpr int kTmemCols = (kACol0 + 32 * kStages <= 256) ? 256 : 512;
-  static_assert(kACol0 + 32 * kStages <= kTmemCols, "TMEM budget");
+  static constexpr int kACols = 64;
+  static constexpr int kTmemCols = (kACol0 + kACols * kStages <= 256) ? 256 : 512;
+  static_assert(kACol0 + kACols * kStages <= kTmemCols, "TMEM budget");
   static constexpr int kLdChunk = (T == 128) ? 32 : 16;   // TMEM columns per load batch
   static_assert(kCols % 16 == 0, "epilogue column chunking");
 };
@@ -215,8 +223,8 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* xs_ring = base;                                  // STAGES * kXsBytes
-  uint8_t* w_ring = base + STAGES * Cfg::kXsBytes;          // STAGES * 12288
-  uint8_t* sc_ring = w_ring + STAGES * kWTileBytes;         // kScSlots slots
+  uint8_t* w_ring = base + STAGES * Cfg::kXsBytes;          // STAGES * 24576
+  uint8_t* sc_ring = w_ring + STAGES * Cfg::kWStageBytes;   // kScSlots slots
   float* red = reinterpret_cast<float*>(base);              // cluster reduction
   GemmCtrl<T>* ctrl = reinterpret_cast<GemmCtrl<T>*>(base + args.ctrl_offset);
 
@@ -229,17 +237,16 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   const int nt = blockIdx.y;            // weight tile
   const int mt = blockIdx.z;            // token tile
   const int M = args.M, N = args.N, K = args.K, gs = args.gs, S = args.split;
-  const int KB = K / kKBlock;
-  const int U = gs > kKBlock ? gs / kKBlock : 1;      // K blocks per split unit
-  const int units = KB / U;
+  const int KB = K / kKBlock;                         // 128-wide weight tiles
+  const int units = K / Cfg::kKStage;                 // stages along K (gs | 256)
   const int u0 = static_cast<int>((static_cast<long long>(ks) * units) / S);
   const int u1 = static_cast<int>((static_cast<long long>(ks + 1) * units) / S);
-  const int kb0 = u0 * U;
-  const int nkb = (u1 - u0) * U;
+  const int kb0 = 2 * u0;                             // first weight tile
+  const int nst = u1 - u0;                            // stages of this CTA
   // gs is a power of two (32..256): group arithmetic uses masks and shifts
   const int gs_log2 = __ffs(gs) - 1;
-  const int g0 = (kb0 * kKBlock) >> gs_log2;
-  const int ngroups = (nkb * kKBlock) >> gs_log2;
+  const int g0 = (u0 * Cfg::kKStage) >> gs_log2;
+  const int ngroups = (nst * Cfg::kKStage) >> gs_log2;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -284,9 +291,9 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       const int n_oct = PARTIALS ? 0 : (ngroups + 7) / 8;
       int next_oct = 0;
       bool ok = true;
-      for (int i = 0; i < nkb && ok; ++i) {
-        // scales: issue octet o at the first K block that touches group 8*o
-        const int lg_first = (i * kKBlock) >> gs_log2;
+      for (int i = 0; i < nst && ok; ++i) {
+        // scales: issue octet o at the first stage that touches group 8*o
+        const int lg_first = (i * Cfg::kKStage) >> gs_log2;
         while (next_oct < n_oct && next_oct * 8 <= lg_first) {
           const int o = next_oct, slot = o % Cfg::kScSlots;
           if (o >= Cfg::kScSlots &&
@@ -312,17 +319,20 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
           break;
         }
         if (args.stall && i == 0) continue;
+        const int kb = kb0 + 2 * i;
+        uint8_t* xs = xs_ring + s * Cfg::kXsBytes;
         mbar_arrive_expect_tx(&ctrl->full[s], Cfg::kStageBytes);
-        tma_load_2d(xs_ring + s * Cfg::kXsBytes, &tmap_x, &ctrl->full[s],
-                    (kb0 + i) * kKBlock, mt * T);
-        bulk_load(w_ring + s * kWTileBytes,
-                  args.wp + (static_cast<size_t>(nt) * KB + kb0 + i) * kWTileBytes,
-                  kWTileBytes, &ctrl->full[s]);
+        tma_load_2d(xs, &tmap_x, &ctrl->full[s], kb * kKBlock, mt * T);
+        tma_load_2d(xs + Cfg::kXsHalf, &tmap_x, &ctrl->full[s], (kb + 1) * kKBlock, mt * T);
+        // tiles (nt, kb) and (nt, kb + 1) are adjacent in the device form
+        bulk_load(w_ring + s * Cfg::kWStageBytes,
+                  args.wp + (static_cast<size_t>(nt) * KB + kb) * kWTileBytes,
+                  Cfg::kWStageBytes, &ctrl->full[s]);
         issued |= 1u << s;
         parity = (parity & ~(1u << s)) | (static_cast<uint32_t>((i / STAGES) & 1) << s);
       }
       if (!ok) record_status(args.status, kStatusTimeout, 0);
-      FLEXQ_ROLE_DONE(0, nkb);
+      FLEXQ_ROLE_DONE(0, nst);
       // every issued copy must land before the CTA may finish
       for (int s = 0; s < STAGES; ++s)
         if ((issued >> s) & 1u) mbar_wait(&ctrl->full[s], (parity >> s) & 1u, lim);
@@ -335,42 +345,36 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     // The issuing thread shares its SM sub-partition with busy unpack and
     // epilogue warps, so every instruction on its path counts: the loop is
     // unrolled over the stages (addresses become constants) and the group
-    // boundaries of the four 32-wide MMAs of a K block come from two 4-bit
-    // masks (indexed by the K block's parity, which matters for gs = 256).
+    // boundaries of the eight 32-wide MMAs of a stage come from two masks
+    // (stages start group-aligned for every gs in 32..256).
     if (lane == 0) {
       FLEXQ_ROLE_CLOCK;
       constexpr uint32_t idesc = idesc_i8(kTileRows, T);
-      uint32_t first_mask[2], last_mask[2];
+      uint32_t first_mask = 0, last_mask = 0;
 #pragma unroll
-      for (int par = 0; par < 2; ++par) {
-        first_mask[par] = last_mask[par] = 0;
-#pragma unroll
-        for (int sub = 0; sub < 4; ++sub) {
-          const int kk = par * kKBlock + sub * 32;    // K-block ranges start group-aligned
-          if ((kk & (gs - 1)) == 0) first_mask[par] |= 1u << sub;
-          if (((kk + 32) & (gs - 1)) == 0) last_mask[par] |= 1u << sub;
-        }
+      for (int sub = 0; sub < 8; ++sub) {
+        if (((sub * 32) & (gs - 1)) == 0) first_mask |= 1u << sub;
+        if (((sub * 32 + 32) & (gs - 1)) == 0) last_mask |= 1u << sub;
       }
       const uint64_t desc0 = smem_desc_k_sw128(smem_u32(xs_ring));
       const uint32_t a_col0 = tmem + Cfg::kACol0;
       uint32_t phase = 0, b = 0;
       int pass = 0;
       bool ok = true;
-      for (int i0 = 0; i0 < nkb && ok; i0 += STAGES) {
+      for (int i0 = 0; i0 < nst && ok; i0 += STAGES) {
 #pragma unroll
         for (int s = 0; s < STAGES; ++s) {
           const int i = i0 + s;
-          if (i >= nkb) break;
+          if (i >= nst) break;
           if (!FLEXQ_WAIT(mbar_wait(&ctrl->full[s], phase, lim)) ||
               !FLEXQ_WAIT(mbar_wait(&ctrl->a_full[s], phase, lim))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t fm = first_mask[i & 1], lm = last_mask[i & 1];
 #pragma unroll
-          for (int sub = 0; sub < 4; ++sub) {
-            const bool first = (fm >> sub) & 1u;
+          for (int sub = 0; sub < 8; ++sub) {
+            const bool first = (first_mask >> sub) & 1u;
             if (first && pass > 0) {
               if (!FLEXQ_WAIT(mbar_wait(&ctrl->p_empty[b], (pass - 1) & 1, lim))) {
                 ok = false;
@@ -378,10 +382,13 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
               }
               tc_fence_after();
             }
-            mma_i8_tmem_a(tmem + Cfg::kPCol0 + b * T, a_col0 + s * 32 + sub * 8,
-                          desc0 + ((s * Cfg::kXsBytes + sub * 32) >> 4), idesc,
-                          first ? 0u : 1u);
-            if ((lm >> sub) & 1u) {
+            // A: weights of this stage in TMEM (8 columns per 32 codes);
+            // B: activation box (sub / 4), 32-byte K step (sub % 4)
+            mma_i8_tmem_a(tmem + Cfg::kPCol0 + b * T, a_col0 + s * Cfg::kACols + sub * 8,
+                          desc0 + ((s * Cfg::kXsBytes + (sub >> 2) * Cfg::kXsHalf +
+                                    (sub & 3) * 32) >> 4),
+                          idesc, first ? 0u : 1u);
+            if ((last_mask >> sub) & 1u) {
               mma_commit(&ctrl->p_full[b]);
               if (++b == Cfg::kPBufs) {
                 b = 0;
@@ -395,7 +402,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         phase ^= 1;
       }
       if (!ok) record_status(args.status, kStatusTimeout, 1);
-      FLEXQ_ROLE_DONE(1, nkb);
+      FLEXQ_ROLE_DONE(1, nst);
       // all issued MMAs must finish before TMEM is released
       mma_commit(&ctrl->done);
       mbar_wait(&ctrl->done, 0, lim);
@@ -407,37 +414,40 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     const int row = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     FLEXQ_ROLE_CLOCK;
-    for (int i = 0; i < nkb; ++i) {
+    for (int i = 0; i < nst; ++i) {
       const int s = i % STAGES;
       if (!FLEXQ_WAIT(warp_wait(&ctrl->full[s], (i / STAGES) & 1, lim))) {
         if (lane == 0) record_status(args.status, kStatusTimeout, 2);
         break;
       }
-      const uint4* src = reinterpret_cast<const uint4*>(w_ring + s * kWTileBytes) + row;
-      uint32_t wa[12], wb[12];
+      // this row's 2 x 96 packed bytes: chunk j of tile t at t*12288 + (j*128 + row)*16
+      const uint4* src = reinterpret_cast<const uint4*>(w_ring + s * Cfg::kWStageBytes) + row;
+      uint32_t w[4][12];
 #pragma unroll
-      for (int j = 0; j < 3; ++j) {
-        const uint4 a = src[j * 128];
-        const uint4 b = src[(j + 3) * 128];
-        wa[4 * j] = a.x; wa[4 * j + 1] = a.y; wa[4 * j + 2] = a.z; wa[4 * j + 3] = a.w;
-        wb[4 * j] = b.x; wb[4 * j + 1] = b.y; wb[4 * j + 2] = b.z; wb[4 * j + 3] = b.w;
+      for (int t = 0; t < 2; ++t) {
+#pragma unroll
+        for (int j = 0; j < 6; ++j) {
+          const uint4 v = src[t * (kWTileBytes / 16) + j * 128];
+          uint32_t* d = &w[2 * t + j / 3][4 * (j % 3)];
+          d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->empty[s]);
-      const int slot = s;                   // free: see GemmCfg
-      tc_fence_after();
-      const uint32_t col = tmem + lane_base + Cfg::kACol0 + slot * 32;
-      uint32_t out[16];
-      unpack48(wa, out);
-      tmem_st16(col, out);
-      unpack48(wb, out);
-      tmem_st16(col + 16, out);
+      tc_fence_after();                     // A slot s is free: see GemmCfg
+      const uint32_t col = tmem + lane_base + Cfg::kACol0 + s * Cfg::kACols;
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        uint32_t out[16];
+        unpack48(w[h], out);
+        tmem_st16(col + 16 * h, out);
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctrl->a_full[slot]);
+      if (lane == 0) mbar_arrive(&ctrl->a_full[s]);
     }
-    if (q == 0 && lane == 0) FLEXQ_ROLE_DONE(2, nkb);
+    if (q == 0 && lane == 0) FLEXQ_ROLE_DONE(2, nst);
   } else {
     // ------------------------------------------------------ epilogue -----
     const int e = warp - 6;

@@ -16,8 +16,9 @@
  *     allocates, frees or retains them.  FP16 buffers are IEEE binary16.
  *   - Matrices are row-major.  M = tokens, N = output channels, K = input
  *     channels, gs = group size along K, G = K / gs.
- *   - Supported shapes: M >= 0 (M == 0 is a no-op), N % 128 == 0, K % 128 == 0,
- *     gs in {32, 64, 128, 256}, K % gs == 0.
+ *   - Supported shapes: M >= 0 (M == 0 is a no-op), N % 128 == 0, K % 256 == 0,
+ *     gs in {32, 64, 128, 256} (K % gs == 0 follows).  Activation
+ *     quantization alone only needs K % gs == 0.
  *   - Every device pointer must be 16-byte aligned.  With M == 0 the
  *     activation-side pointers are not read and may be NULL.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls

@@ -49,7 +49,8 @@ def test_packed_size(L):
     assert L.flexq_weight_packed_bytes(28672, 8192, 32) == 28672 * 8192 * 3 // 4
     assert L.flexq_weight_packed_bytes(100, 4096, 128) == 0        # N % 128
     assert L.flexq_weight_packed_bytes(128, 4096, 48) == 0         # bad gs
-    assert L.flexq_weight_packed_bytes(128, 192, 64) == 0          # K % 128
+    assert L.flexq_weight_packed_bytes(128, 192, 64) == 0          # K % 256
+    assert L.flexq_weight_packed_bytes(128, 384, 128) == 0         # K % 256
 
 
 FAKE = ctypes.c_void_p(1 << 20)          # never dereferenced: validation fails first
