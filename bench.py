@@ -369,7 +369,7 @@ def run_flexq(args, rank, world):
     traffic = profiled_traffic()
     result = {
         "metric": METRIC,
-        "value": round(aggregate(ops, world, t_max_s) / 1e12, 3),
+        "value": round(aggregate(ops * args.steps, world, t_max_s) / 1e12, 3),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
@@ -488,7 +488,7 @@ def run_e2e(W, args, device, world):
     torch.cuda.synchronize(device)
     t_max = max_over_ranks(t0.elapsed_time(t1) / 1e3, device)
     ops = step_ops(W.ms, [(n, N, K) for (n, N, K, _, _) in W.w])
-    return {"value": round(aggregate(ops, world, t_max) / 1e12, 3), "unit": UNIT,
+    return {"value": round(aggregate(ops * args.steps, world, t_max) / 1e12, 3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(t_max * 1e3 / args.steps, 4)}
 

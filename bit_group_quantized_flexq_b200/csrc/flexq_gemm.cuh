@@ -39,6 +39,7 @@
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "flexq_ptx.cuh"
 
@@ -342,64 +343,84 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     __syncwarp();
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA -----
-    // The issuing thread shares its SM sub-partition with busy unpack and
-    // epilogue warps, so every instruction on its path counts: the loop is
-    // unrolled over the stages (addresses become constants) and the group
-    // boundaries of the eight 32-wide MMAs of a stage come from two masks
-    // (stages start group-aligned for every gs in 32..256).
+    // On the issuing thread a tcgen05.mma is cheap only inside a straight
+    // run of MMAs: any branch, predicated tcgen05 op or commit between two
+    // MMAs waits for the previous one to be taken by the tensor pipe, which
+    // roughly doubles the cost per MMA. So the eight 32-wide MMAs of a stage
+    // are one straight run: the group size is a compile-time constant here
+    // (group boundaries, accumulate flags and commit points fixed), and a
+    // stage waits on two barriers only, both before its first MMA:
+    //   a_full[s]  the unpack warps stored the weights of the stage in TMEM;
+    //              they do so after observing full[s], so the activations the
+    //              TMA brought into shared memory are in place too;
+    //   p_empty    with at least twice as many partial buffers as groups
+    //              per stage: the buffer of the stage's last group, released
+    //              by the epilogue; it releases buffers in order, so every
+    //              earlier buffer is free as well, and the epilogue still
+    //              has a whole stage of groups to work on meanwhile;
+    //              otherwise the buffer of the first group only, and each
+    //              later group of the stage waits for its own buffer (one
+    //              wait at stage start would keep the MMAs of the stage
+    //              from overlapping the epilogue of the previous one).
     if (lane == 0) {
       FLEXQ_ROLE_CLOCK;
-      constexpr uint32_t idesc = idesc_i8(kTileRows, T);
-      uint32_t first_mask = 0, last_mask = 0;
-#pragma unroll
-      for (int sub = 0; sub < 8; ++sub) {
-        if (((sub * 32) & (gs - 1)) == 0) first_mask |= 1u << sub;
-        if (((sub * 32 + 32) & (gs - 1)) == 0) last_mask |= 1u << sub;
-      }
       const uint64_t desc0 = smem_desc_k_sw128(smem_u32(xs_ring));
       const uint32_t a_col0 = tmem + Cfg::kACol0;
-      uint32_t phase = 0, b = 0;
-      int pass = 0;
-      bool ok = true;
-      for (int i0 = 0; i0 < nst && ok; i0 += STAGES) {
+      auto run = [&](auto gs_c) -> bool {
+        constexpr int GS = decltype(gs_c)::value;
+        constexpr int G = Cfg::kKStage / GS;            // groups per stage
+        constexpr int SPG = GS / 32;                     // MMAs per group
+        constexpr int NB = Cfg::kPBufs;
+        constexpr int LOG_NB = (NB == 4) ? 2 : 1;
+        constexpr bool kBatch = NB >= 2 * G;
+        constexpr int W0 = kBatch ? G : 1;              // groups the stage-start wait covers
+        constexpr uint32_t idesc = idesc_i8(kTileRows, T);
+        static_assert(NB == (1 << LOG_NB), "partial buffers: power of two");
+        uint32_t g = 0, phase = 0;
+        for (int i0 = 0; i0 < nst; i0 += STAGES) {
 #pragma unroll
-        for (int s = 0; s < STAGES; ++s) {
-          const int i = i0 + s;
-          if (i >= nst) break;
-          if (!FLEXQ_WAIT(mbar_wait(&ctrl->full[s], phase, lim)) ||
-              !FLEXQ_WAIT(mbar_wait(&ctrl->a_full[s], phase, lim))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+          for (int s = 0; s < STAGES; ++s) {
+            if (i0 + s >= nst) return true;
+            const uint32_t gl = g + W0 - 1;
+            // use u of a buffer waits for the release of use u - 1: parity
+            // (u & 1) ^ 1, which a fresh barrier reports complete for u = 0
+            if (!FLEXQ_WAIT(mbar_wait(&ctrl->a_full[s], phase, lim)) ||
+                !FLEXQ_WAIT(mbar_wait(&ctrl->p_empty[gl & (NB - 1)], ((gl >> LOG_NB) & 1u) ^ 1u, lim)))
+              return false;
+            tc_fence_after();
 #pragma unroll
-          for (int sub = 0; sub < 8; ++sub) {
-            const bool first = (first_mask >> sub) & 1u;
-            if (first && pass > 0) {
-              if (!FLEXQ_WAIT(mbar_wait(&ctrl->p_empty[b], (pass - 1) & 1, lim))) {
-                ok = false;
-                break;
+            for (int j = 0; j < G; ++j) {
+              const uint32_t gj = g + j, buf = gj & (NB - 1);
+              if (j >= W0) {
+                if (!FLEXQ_WAIT(mbar_wait(&ctrl->p_empty[buf], ((gj >> LOG_NB) & 1u) ^ 1u, lim)))
+                  return false;
+                tc_fence_after();
               }
-              tc_fence_after();
-            }
-            // A: weights of this stage in TMEM (8 columns per 32 codes);
-            // B: activation box (sub / 4), 32-byte K step (sub % 4)
-            mma_i8_tmem_a(tmem + Cfg::kPCol0 + b * T, a_col0 + s * Cfg::kACols + sub * 8,
-                          desc0 + ((s * Cfg::kXsBytes + (sub >> 2) * Cfg::kXsHalf +
-                                    (sub & 3) * 32) >> 4),
-                          idesc, first ? 0u : 1u);
-            if ((last_mask >> sub) & 1u) {
-              mma_commit(&ctrl->p_full[b]);
-              if (++b == Cfg::kPBufs) {
-                b = 0;
-                ++pass;
+#pragma unroll
+              for (int k = 0; k < SPG; ++k) {
+                const int sub = j * SPG + k;
+                // A: weights of this stage in TMEM (8 columns per 32 codes);
+                // B: activation box (sub / 4), 32-byte K step (sub % 4)
+                mma_i8_tmem_a(tmem + Cfg::kPCol0 + buf * T, a_col0 + s * Cfg::kACols + sub * 8,
+                              desc0 + ((s * Cfg::kXsBytes + (sub >> 2) * Cfg::kXsHalf +
+                                        (sub & 3) * 32) >> 4),
+                              idesc, k == 0 ? 0u : 1u);
               }
+              mma_commit(&ctrl->p_full[buf]);
             }
+            mma_commit(&ctrl->empty[s]);     // frees smem stage s and A slot s
+            g += G;
           }
-          if (!ok) break;
-          mma_commit(&ctrl->empty[s]);     // frees smem stage s and A slot s
+          phase ^= 1;
         }
-        phase ^= 1;
+        return true;
+      };
+      bool ok;
+      switch (gs) {
+        case 32: ok = run(std::integral_constant<int, 32>{}); break;
+        case 64: ok = run(std::integral_constant<int, 64>{}); break;
+        case 128: ok = run(std::integral_constant<int, 128>{}); break;
+        default: ok = run(std::integral_constant<int, 256>{}); break;
       }
       if (!ok) record_status(args.status, kStatusTimeout, 1);
       FLEXQ_ROLE_DONE(1, nst);
