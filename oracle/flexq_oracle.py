@@ -34,8 +34,9 @@ Readings where the pages are silent (each listed in the design notes):
   and all codes 0;
 * the 6-bit weight container packs 4 codes into 3 bytes, little endian,
   code i in bits [6i, 6i+6) as 6-bit two's complement ("canonical form");
-  the device form is a fixed permutation of those bytes into 128-row tiles
-  (``reorder_to_device_form``);
+  the device form keeps 4 codes per 3 bytes but places twelve of every
+  sixteen codes byte-aligned (``pack_block_words``) and tiles the rows into
+  128 x 128-code tiles (``pack_device_form``);
 * Y is formed in FP64 from the exact integer partials and the exact FP16
   scales, then rounded once to FP16 (round-to-nearest-even).
 
@@ -138,34 +139,80 @@ def unpack_canonical(packed, K):
 
 
 # --------------------------------------------------------------------------
-# device form: canonical bytes permuted into 128-row x 128-k tiles
+# device form: the 6-bit codes of 16 consecutive k in 12 bytes, laid out so
+# that twelve codes sit byte-aligned; rows tiled into 128 x 128-code tiles
 # --------------------------------------------------------------------------
 TILE_ROWS = 128          # weight rows per tile
 TILE_K = 128             # codes per row per tile (96 packed bytes)
 CHUNK = 16               # bytes per chunk; 6 chunks per row per tile
+BLOCK = 16               # codes per 12-byte block
 
 
-def reorder_to_device_form(packed, N, K):
-    """Permute canonical packed bytes [N, 3K/4] into the device form.
+def pack_block_words(codes16):
+    """The three 32-bit words of one 16-code block.
 
-    The device form is a flat byte array of (N/128) * (K/128) tiles of 12288
-    bytes; tile (nt, kb) holds rows nt*128 .. nt*128+127 and codes
-    kb*128 .. kb*128+127.  Inside a tile the 96 bytes of each row are cut into
-    six 16-byte chunks and stored chunk-major: byte b of chunk j of row r sits
-    at offset (j*128 + r)*16 + b.  In other words, device byte
-    [nt][kb][j][r][b] = canonical byte [nt*128 + r][kb*96 + 16*j + b].
+    codes16: int array [..., 16] of 6-bit codes in [-32, 31]; u_j = c_j & 63.
+    For word i in {0, 1, 2} and byte t in {0, 1, 2, 3}:
+      bits [8t+2, 8t+8) hold u_{4i+t}                (twelve aligned codes),
+      bits [8t,   8t+2) hold bits [2i, 2i+2) of u_{12+t} (the four codes
+                                                     12..15, two bits per word).
+    Four codes per three bytes, every field two's complement.
     """
+    c = np.asarray(codes16)
+    assert c.shape[-1] == BLOCK
+    assert c.min(initial=0) >= -32 and c.max(initial=0) <= 31
+    u = (c.astype(np.int64) & 0x3F).astype(np.uint64)
+    words = np.zeros(c.shape[:-1] + (3,), dtype=np.uint64)
+    for i in range(3):
+        for t in range(4):
+            aligned = u[..., 4 * i + t] << np.uint64(8 * t + 2)
+            spread = ((u[..., 12 + t] >> np.uint64(2 * i)) & np.uint64(3)) << np.uint64(8 * t)
+            words[..., i] |= aligned | spread
+    return words.astype(np.uint32)
+
+
+def unpack_block_words(words):
+    """Inverse of pack_block_words: uint32 [..., 3] -> int8 codes [..., 16]."""
+    w = np.asarray(words).astype(np.uint64)
+    assert w.shape[-1] == 3
+    u = np.zeros(w.shape[:-1] + (BLOCK,), dtype=np.int64)
+    for i in range(3):
+        for t in range(4):
+            u[..., 4 * i + t] = (w[..., i] >> np.uint64(8 * t + 2)) & np.uint64(0x3F)
+            piece = (w[..., i] >> np.uint64(8 * t)) & np.uint64(3)
+            u[..., 12 + t] |= (piece << np.uint64(2 * i)).astype(np.int64)
+    signed = u - 64 * (u >= 32)
+    return signed.astype(np.int8)
+
+
+def pack_device_form(codes):
+    """6-bit codes [N, K] (N % 128 == 0, K % 128 == 0) -> device-form bytes.
+
+    Each row is cut into 16-code blocks, block b of row n becoming the 12
+    little-endian bytes of pack_block_words(codes[n, 16b:16b+16]); a row's 128
+    codes of K-block kb are its 96 bytes kb*96 .. kb*96+95.  Those 96 bytes are
+    cut into six 16-byte chunks and tiled: tile (nt, kb) (rows nt*128 ..
+    nt*128+127, codes kb*128 .. kb*128+127) is 12288 contiguous bytes at
+    offset (nt*(K/128) + kb) * 12288, and byte b of chunk j of row r sits at
+    offset (j*128 + r)*16 + b inside the tile.
+    """
+    codes = np.asarray(codes)
+    N, K = codes.shape
     assert N % TILE_ROWS == 0 and K % TILE_K == 0
+    words = pack_block_words(codes.reshape(N, K // BLOCK, BLOCK))      # [N, K/16, 3]
+    row_bytes = words.astype("<u4").view(np.uint8).reshape(N, 3 * K // 4)
     NT, KB = N // TILE_ROWS, K // TILE_K
-    v = np.asarray(packed, dtype=np.uint8).reshape(NT, TILE_ROWS, KB, 6, CHUNK)
+    v = row_bytes.reshape(NT, TILE_ROWS, KB, 6, CHUNK)
     return np.ascontiguousarray(v.transpose(0, 2, 3, 1, 4)).reshape(-1)
 
 
-def device_form_to_canonical(dev, N, K):
-    """Inverse permutation of reorder_to_device_form."""
+def unpack_device_form(dev, N, K):
+    """Inverse of pack_device_form: device-form bytes -> int8 codes [N, K]."""
     NT, KB = N // TILE_ROWS, K // TILE_K
     v = np.asarray(dev, dtype=np.uint8).reshape(NT, KB, 6, TILE_ROWS, CHUNK)
-    return np.ascontiguousarray(v.transpose(0, 3, 1, 2, 4)).reshape(N, 3 * K // 4)
+    row_bytes = np.ascontiguousarray(v.transpose(0, 3, 1, 2, 4)).reshape(N, 3 * K // 4)
+    words = row_bytes.view("<u4").reshape(N, K // BLOCK, 3)
+    return unpack_block_words(words).reshape(N, K)
 
 
 # --------------------------------------------------------------------------

@@ -18,14 +18,14 @@ def oracle_weight_device_form(w16, gs):
     """Oracle codes, scales and device-form bytes for an FP16 weight [N, K]."""
     qw, sw = orc.quantize_weight(w16, gs)
     N, K = w16.shape
-    dev = orc.reorder_to_device_form(orc.pack_canonical(qw), N, K)
+    dev = orc.pack_device_form(qw)
     return qw, sw, dev
 
 
 def upload_codes_as_weights(qw):
     """Pack arbitrary 6-bit codes [N, K] (oracle packing) into a device buffer."""
     N, K = qw.shape
-    dev = orc.reorder_to_device_form(orc.pack_canonical(qw), N, K)
+    dev = orc.pack_device_form(qw)
     return torch.from_numpy(dev.copy()).cuda()
 
 

@@ -253,27 +253,72 @@ def test_pack_unpack_identity_exhaustive():
     assert np.unique(w).size == 64 ** 4
 
 
-def test_device_form_is_a_permutation_with_the_stated_positions():
+def _block_codes(spec):
+    c = np.zeros(16, dtype=np.int8)
+    if spec == "all -1":
+        c[:] = -1
+    else:
+        for j, v in spec.items():
+            c[int(j)] = v
+    return c
+
+
+def test_device_block_hand_worked_cases(golden_dir):
+    g = _golden("device_form_cases.json", golden_dir)
+    for case in g["cases"]:
+        codes = _block_codes(case["codes"])
+        words = orc.pack_block_words(codes)
+        assert words.astype("<u4").tobytes().hex() == case["bytes"], case
+        assert np.array_equal(orc.unpack_block_words(words), codes)
+
+
+def test_device_block_is_a_bit_permutation():
+    # setting one bit of one code's 6-bit field sets exactly one bit of the
+    # block, and the 96 (code, bit) pairs land on 96 distinct bits: the block
+    # is a bijection of 16 six-bit fields onto 96 bits
+    seen = set()
+    for j in range(16):
+        for bit in range(6):
+            u = 1 << bit
+            c = np.zeros(16, dtype=np.int8)
+            c[j] = u - 64 if u >= 32 else u
+            w = orc.pack_block_words(c).astype(np.uint64)
+            value = int(w[0]) | (int(w[1]) << 32) | (int(w[2]) << 64)
+            assert bin(value).count("1") == 1, (j, bit)
+            seen.add(value.bit_length() - 1)
+    assert seen == set(range(96))
+
+
+def test_device_block_roundtrip_every_value_at_every_position():
+    rng = np.random.default_rng(4)
+    base = rng.integers(-32, 32, (64, 16)).astype(np.int8)
+    for j in range(16):
+        c = base.copy()
+        c[:, j] = np.arange(-32, 32, dtype=np.int8)
+        assert np.array_equal(orc.unpack_block_words(orc.pack_block_words(c)), c)
+
+
+def test_device_form_tile_positions():
     N, K = 256, 384
     rng = np.random.default_rng(9)
     codes = rng.integers(-32, 32, (N, K)).astype(np.int8)
-    canon = orc.pack_canonical(codes)
-    dev = orc.reorder_to_device_form(canon, N, K)
-    assert dev.size == canon.size
-    assert np.array_equal(orc.device_form_to_canonical(dev, N, K), canon)
-    # spot-check the stated position formula with plain index arithmetic
+    dev = orc.pack_device_form(codes)
+    assert dev.size == N * K * 3 // 4
+    assert np.array_equal(orc.unpack_device_form(dev, N, K), codes)
+    # spot-check the stated position formula with plain index arithmetic:
+    # row n, block b (codes 16b..16b+15) -> row byte 12b + 4i + t of word i
     KB = K // 128
-    for (n, cb) in [(0, 0), (1, 0), (127, 95), (128, 96), (200, 150), (255, 287)]:
-        nt, r = divmod(n, 128)
-        kb, within = divmod(cb, 96)
-        j, b = divmod(within, 16)
-        off = ((nt * KB + kb) * 6 + j) * 128 * 16 + r * 16 + b
-        assert dev[off] == canon[n, cb]
-    # distinct labels land in distinct places
-    labels = np.arange(N * K * 3 // 4, dtype=np.int64).reshape(N, -1)
-    NT = N // 128
-    moved = labels.reshape(NT, 128, KB, 6, 16).transpose(0, 2, 3, 1, 4).reshape(-1)
-    assert np.unique(moved).size == moved.size
+    for n in (0, 1, 127, 128, 200, 255):
+        for b in (0, 5, 7, 8, 15, 23):
+            words = orc.pack_block_words(codes[n, 16 * b:16 * b + 16])
+            row_bytes = words.astype("<u4").tobytes()
+            for pos in range(12):
+                cb = 12 * b + pos                     # byte index within the row
+                nt, r = divmod(n, 128)
+                kb, within = divmod(cb, 96)
+                j, byte = divmod(within, 16)
+                off = ((nt * KB + kb) * 6 + j) * 128 * 16 + r * 16 + byte
+                assert dev[off] == row_bytes[pos], (n, b, pos)
 
 
 # ------------------------------------------------------------ GEMM ----------
