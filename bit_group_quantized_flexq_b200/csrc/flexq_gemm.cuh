@@ -15,21 +15,21 @@
 // output tile and reduces through distributed shared memory).
 //
 // The pipeline advances in stages of 256 codes of K (two 128 x 128 weight
-// tiles), which halves the barrier traffic per byte against one tile per
-// stage.
+// tiles).
 //
 // Warp roles (all pipeline waits are bounded, see mbar_wait):
 //   warp 0      producer: per stage, two TMA boxes of the int8 activations
 //               (T rows x 128 B each, 128-byte swizzle) and one 24576-byte
 //               bulk copy of two consecutive packed weight tiles into a
-//               STAGES-deep ring; per 8 groups, the group scales;
+//               STAGES-deep shared-memory ring; per 8 groups, the group
+//               scales;
 //   warp 1      TMEM allocator and MMA issuer: 8 MMAs (K = 32 each) per
 //               stage into the int32 partial buffer of the current group
-//               (kPBufs buffers of T columns), commits per group;
+//               (kPBufs buffers of T columns), one commit per group;
 //   warps 2..5  unpack: each thread owns one weight row, turns its 192 packed
-//               bytes into 256 int8 codes (code * 4, the 6-bit field in the
-//               top of each byte) and stores them into the TMEM A slot of
-//               the stage (64 columns per stage);
+//               bytes into 256 int8 codes (code * 4: the 6-bit field in the
+//               top of each byte) and stores them into a TMEM "A" slot
+//               (kASlots slots of 64 columns);
 //   warps 6..   epilogue: per group, load the int32 partials from TMEM,
 //               release the buffer, and accumulate
 //               acc += float(P) * (sw[n,g]/4 * sa[m,g]) in FP32 registers;
@@ -63,9 +63,12 @@ struct GemmArgs {
 
 template <int T>
 struct GemmCfg {
-  static constexpr int kEpiWarps = (T <= 32) ? 4 : 8;
+  // each epilogue warp owns one TMEM lane quarter (32 weight rows) and kCols
+  // tokens; T = 128 uses 16 epilogue warps so that four warps per scheduler
+  // hide the latency of the TMEM loads and conversions
+  static constexpr int kCols = T < 32 ? T : 32;
+  static constexpr int kEpiWarps = 4 * (T / kCols);
   static constexpr int kThreads = (6 + kEpiWarps) * 32;
-  static constexpr int kCols = T / (kEpiWarps / 4);      // tokens per epi warp
   static constexpr int kStages = (T == 64) ? 2 : 3;
   static constexpr int kMinBlocks = (T <= 64) ? 2 : 1;
   static constexpr int kMaxSplit = (T == 16) ? 8 : (T == 32) ? 6 : (T == 64) ? 4 : 2;
@@ -81,26 +84,28 @@ struct GemmCfg {
   static constexpr int kScSaBytes = 8 * T * 2;
   static constexpr int kScSlotBytes = kScSaBytes + 8 * 128 * 2;
   static constexpr int kMainBytes = kStages * kStageBytes + kScSlots * kScSlotBytes;
-  // TMEM: int32 partial buffers (one per group in flight), then one A slot
-  // (64 columns = 256 int8 codes per row) per shared-memory stage.  A slot s
-  // is only rewritten for stage i after the producer refilled stage s for
-  // i, which it does only after the MMAs of stage i - STAGES (the previous
-  // user of slot s) have completed, so the slot needs no barrier of its own.
-  static constexpr int kPBufs = (T == 16) ? 4 : 2;
+  // TMEM: int32 partial buffers (one per group in flight), then the A slots
+  // (64 columns = 256 int8 codes per row each).  Two CTAs share an SM for
+  // T <= 64, so those stay within 256 columns; T = 128 takes all 512 for
+  // three partial buffers and two A slots.
+  static constexpr int kPBufs = (T == 16) ? 4 : (T == 128) ? 3 : 2;
+  static constexpr int kASlots = (T == 128) ? 2 : kStages;
   static constexpr int kPCol0 = 0;
   static constexpr int kACol0 = kPBufs * T;
   static constexpr int kACols = 64;
-  static constexpr int kTmemCols = (kACol0 + kACols * kStages <= 256) ? 256 : 512;
-  static_assert(kACol0 + kACols * kStages <= kTmemCols, "TMEM budget");
-  static constexpr int kLdChunk = (T == 128) ? 32 : 16;   // TMEM columns per load batch
-  static_assert(kCols % 16 == 0, "epilogue column chunking");
+  static constexpr int kTmemCols = (kACol0 + kACols * kASlots <= 256) ? 256 : 512;
+  static_assert(kACol0 + kACols * kASlots <= kTmemCols, "TMEM budget");
+  static_assert(kMinBlocks == 1 || kTmemCols <= 256, "two CTAs per SM share 512 columns");
+  static constexpr int kLdChunk = (T == 64) ? 16 : kCols;   // TMEM columns per load batch
+  static_assert(kCols % kLdChunk == 0 && kLdChunk % 16 == 0, "epilogue column chunking");
 };
 
 template <int T>
 struct GemmCtrl {
   uint64_t full[GemmCfg<T>::kStages];
   uint64_t empty[GemmCfg<T>::kStages];
-  uint64_t a_full[GemmCfg<T>::kStages];
+  uint64_t a_full[GemmCfg<T>::kASlots];
+  uint64_t a_empty[GemmCfg<T>::kASlots];
   uint64_t p_full[GemmCfg<T>::kPBufs];
   uint64_t p_empty[GemmCfg<T>::kPBufs];
   uint64_t s_full[GemmCfg<T>::kScSlots];
@@ -110,6 +115,19 @@ struct GemmCtrl {
   uint32_t pad;
   // per epilogue warp: its tokens' activation scales of the current octet, FP32
   alignas(16) float sa[GemmCfg<T>::kEpiWarps][8][GemmCfg<T>::kCols];
+};
+
+// A ring position: index into a ring of R slots and the parity of the
+// current round; advancing past the last slot flips the parity.
+template <int R>
+struct RingPos {
+  uint32_t idx = 0, phase = 0;
+  __device__ __forceinline__ void next() {
+    const uint32_t n = idx + 1;
+    const uint32_t wrap = (n == static_cast<uint32_t>(R)) ? 1u : 0u;
+    idx = wrap ? 0u : n;
+    phase ^= wrap;
+  }
 };
 
 // Optional pipeline trace (compile with -DFLEXQ_TRACE).  Every CTA records
@@ -183,35 +201,28 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
   return ok;
 }
 
-// Four 6-bit codes in the low 24 bits of q (bits above 23 ignored) -> four
-// int8 lanes holding code * 4 (the 6-bit two's-complement field sits in bits
-// [7:2] of each byte).
-__device__ __forceinline__ uint32_t expand_quad(uint32_t q) {
-  const uint32_t t = (q & 0x0000FFFFu) | ((q << 4) & 0xFFFF0000u);
-  return ((t << 2) & 0x00FC00FCu) | ((t << 4) & 0xFC00FC00u);
+// One 16-code block of the device form (three words, see weight_pack_kernel)
+// -> four int8x4 words in k order, each byte code * 4.  Bytes of w0..w2 hold
+// codes 0..11 in their bits [7:2]; their bits [1:0] hold the 2-bit pieces of
+// codes 12..15 (w0: bits 1:0 of the code, w1: bits 3:2, w2: bits 5:4).  The
+// pieces occupy disjoint bits of each byte, so adding them cannot carry.
+__device__ __forceinline__ void unpack_block(uint32_t w0, uint32_t w1, uint32_t w2,
+                                             uint32_t* out) {
+  out[0] = w0 & 0xFCFCFCFCu;
+  out[1] = w1 & 0xFCFCFCFCu;
+  out[2] = w2 & 0xFCFCFCFCu;
+  const uint32_t p0 = w0 & 0x03030303u, p1 = w1 & 0x03030303u, p2 = w2 & 0x03030303u;
+  out[3] = ((p2 * 4u + p1) * 4u + p0) * 4u;
 }
 
-// 12 canonical packed words (16 quads, 64 codes) -> 16 int8x4 words.
-__device__ __forceinline__ void unpack48(const uint32_t (&w)[12],
-                                         uint32_t (&out)[16]) {
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const uint32_t w0 = w[3 * t], w1 = w[3 * t + 1], w2 = w[3 * t + 2];
-    out[4 * t + 0] = expand_quad(w0);
-    out[4 * t + 1] = expand_quad(__funnelshift_r(w0, w1, 24));
-    out[4 * t + 2] = expand_quad(__funnelshift_r(w1, w2, 16));
-    out[4 * t + 3] = expand_quad(w2 >> 8);
+template <int CH>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[CH]) {
+  static_assert(CH == 16 || CH == 32, "16 or 32 columns per load");
+  if constexpr (CH == 32) {
+    tmem_ld32(taddr, r);
+  } else {
+    tmem_ld16(taddr, r);
   }
-}
-
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, "
-      "%7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
-      "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]),
-      "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
 }
 
 template <int T, bool PARTIALS>
@@ -221,6 +232,8 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
                      const __grid_constant__ CUtensorMap tmap_sw, const GemmArgs args) {
   using Cfg = GemmCfg<T>;
   constexpr int STAGES = Cfg::kStages;
+  constexpr int ASLOTS = Cfg::kASlots;
+  constexpr int NB = Cfg::kPBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* xs_ring = base;                                  // STAGES * kXsBytes
@@ -254,8 +267,11 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       mbar_init(&ctrl->full[s], 1);
       mbar_init(&ctrl->empty[s], 4 + 1);     // 4 unpack warps + MMA commit
     }
-    for (int s = 0; s < STAGES; ++s) mbar_init(&ctrl->a_full[s], 4);
-    for (int b = 0; b < Cfg::kPBufs; ++b) {
+    for (int a = 0; a < ASLOTS; ++a) {
+      mbar_init(&ctrl->a_full[a], 4);        // 4 unpack warps
+      mbar_init(&ctrl->a_empty[a], 1);       // MMA commit
+    }
+    for (int b = 0; b < NB; ++b) {
       mbar_init(&ctrl->p_full[b], 1);
       mbar_init(&ctrl->p_empty[b], Cfg::kEpiWarps);
     }
@@ -345,73 +361,68 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     // ----------------------------------------------------------- MMA -----
     // On the issuing thread a tcgen05.mma is cheap only inside a straight
     // run of MMAs: any branch, predicated tcgen05 op or commit between two
-    // MMAs waits for the previous one to be taken by the tensor pipe, which
-    // roughly doubles the cost per MMA. So the eight 32-wide MMAs of a stage
-    // are one straight run: the group size is a compile-time constant here
-    // (group boundaries, accumulate flags and commit points fixed), and a
-    // stage waits on two barriers only, both before its first MMA:
-    //   a_full[s]  the unpack warps stored the weights of the stage in TMEM;
-    //              they do so after observing full[s], so the activations the
-    //              TMA brought into shared memory are in place too;
+    // MMAs waits for the previous one to be taken by the tensor pipe.  So the
+    // MMAs of a group are one straight run (the group size is a compile-time
+    // constant here), and the waits sit before a group's first MMA:
+    //   a_full[a]  the unpack warps stored the stage's weights in A slot a;
+    //              they do so after observing full[s], so the activations
+    //              the TMA brought into shared memory are in place too;
     //   p_empty    with at least twice as many partial buffers as groups
-    //              per stage: the buffer of the stage's last group, released
-    //              by the epilogue; it releases buffers in order, so every
-    //              earlier buffer is free as well, and the epilogue still
-    //              has a whole stage of groups to work on meanwhile;
-    //              otherwise the buffer of the first group only, and each
-    //              later group of the stage waits for its own buffer (one
-    //              wait at stage start would keep the MMAs of the stage
-    //              from overlapping the epilogue of the previous one).
+    //              per stage, one wait at the stage start for the buffer of
+    //              the stage's last group (the epilogue releases buffers in
+    //              order, so the earlier ones are free too, and it still has
+    //              a whole stage of groups to work on meanwhile); otherwise
+    //              each group waits for its own buffer.
     if (lane == 0) {
       FLEXQ_ROLE_CLOCK;
       const uint64_t desc0 = smem_desc_k_sw128(smem_u32(xs_ring));
-      const uint32_t a_col0 = tmem + Cfg::kACol0;
       auto run = [&](auto gs_c) -> bool {
         constexpr int GS = decltype(gs_c)::value;
         constexpr int G = Cfg::kKStage / GS;            // groups per stage
         constexpr int SPG = GS / 32;                     // MMAs per group
-        constexpr int NB = Cfg::kPBufs;
-        constexpr int LOG_NB = (NB == 4) ? 2 : 1;
         constexpr bool kBatch = NB >= 2 * G;
-        constexpr int W0 = kBatch ? G : 1;              // groups the stage-start wait covers
         constexpr uint32_t idesc = idesc_i8(kTileRows, T);
-        static_assert(NB == (1 << LOG_NB), "partial buffers: power of two");
-        uint32_t g = 0, phase = 0;
-        for (int i0 = 0; i0 < nst; i0 += STAGES) {
+        RingPos<STAGES> st;
+        RingPos<ASLOTS> as;
+        RingPos<NB> pb;                                  // buffer of the next group
+        for (int i = 0; i < nst; ++i) {
+          if (!FLEXQ_WAIT(mbar_wait(&ctrl->a_full[as.idx], as.phase, lim))) return false;
+          if constexpr (kBatch) {
+            RingPos<NB> last = pb;
 #pragma unroll
-          for (int s = 0; s < STAGES; ++s) {
-            if (i0 + s >= nst) return true;
-            const uint32_t gl = g + W0 - 1;
+            for (int j = 1; j < G; ++j) last.next();
             // use u of a buffer waits for the release of use u - 1: parity
             // (u & 1) ^ 1, which a fresh barrier reports complete for u = 0
-            if (!FLEXQ_WAIT(mbar_wait(&ctrl->a_full[s], phase, lim)) ||
-                !FLEXQ_WAIT(mbar_wait(&ctrl->p_empty[gl & (NB - 1)], ((gl >> LOG_NB) & 1u) ^ 1u, lim)))
+            if (!FLEXQ_WAIT(mbar_wait(&ctrl->p_empty[last.idx], last.phase ^ 1u, lim)))
               return false;
-            tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < G; ++j) {
-              const uint32_t gj = g + j, buf = gj & (NB - 1);
-              if (j >= W0) {
-                if (!FLEXQ_WAIT(mbar_wait(&ctrl->p_empty[buf], ((gj >> LOG_NB) & 1u) ^ 1u, lim)))
-                  return false;
-                tc_fence_after();
-              }
-#pragma unroll
-              for (int k = 0; k < SPG; ++k) {
-                const int sub = j * SPG + k;
-                // A: weights of this stage in TMEM (8 columns per 32 codes);
-                // B: activation box (sub / 4), 32-byte K step (sub % 4)
-                mma_i8_tmem_a(tmem + Cfg::kPCol0 + buf * T, a_col0 + s * Cfg::kACols + sub * 8,
-                              desc0 + ((s * Cfg::kXsBytes + (sub >> 2) * Cfg::kXsHalf +
-                                        (sub & 3) * 32) >> 4),
-                              idesc, k == 0 ? 0u : 1u);
-              }
-              mma_commit(&ctrl->p_full[buf]);
-            }
-            mma_commit(&ctrl->empty[s]);     // frees smem stage s and A slot s
-            g += G;
           }
-          phase ^= 1;
+          tc_fence_after();
+          const uint32_t a_col = tmem + Cfg::kACol0 + as.idx * Cfg::kACols;
+          const uint64_t b_desc = desc0 + ((st.idx * Cfg::kXsBytes) >> 4);
+#pragma unroll
+          for (int j = 0; j < G; ++j) {
+            if constexpr (!kBatch) {
+              if (!FLEXQ_WAIT(mbar_wait(&ctrl->p_empty[pb.idx], pb.phase ^ 1u, lim)))
+                return false;
+              tc_fence_after();
+            }
+            const uint32_t d_col = tmem + Cfg::kPCol0 + pb.idx * T;
+#pragma unroll
+            for (int k = 0; k < SPG; ++k) {
+              const int sub = j * SPG + k;
+              // A: weights of this stage in TMEM (8 columns per 32 codes);
+              // B: activation box (sub / 4), 32-byte K step (sub % 4)
+              mma_i8_tmem_a(d_col, a_col + sub * 8,
+                            b_desc + (((sub >> 2) * Cfg::kXsHalf + (sub & 3) * 32) >> 4), idesc,
+                            k == 0 ? 0u : 1u);
+            }
+            mma_commit(&ctrl->p_full[pb.idx]);
+            pb.next();
+          }
+          mma_commit(&ctrl->empty[st.idx]);     // frees the smem stage
+          mma_commit(&ctrl->a_empty[as.idx]);   // frees the A slot
+          st.next();
+          as.next();
         }
         return true;
       };
@@ -435,42 +446,46 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     const int row = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     FLEXQ_ROLE_CLOCK;
+    RingPos<STAGES> st;
+    RingPos<ASLOTS> as;
     for (int i = 0; i < nst; ++i) {
-      const int s = i % STAGES;
-      if (!FLEXQ_WAIT(warp_wait(&ctrl->full[s], (i / STAGES) & 1, lim))) {
+      if (!FLEXQ_WAIT(warp_wait(&ctrl->full[st.idx], st.phase, lim)) ||
+          !FLEXQ_WAIT(warp_wait(&ctrl->a_empty[as.idx], as.phase ^ 1u, lim))) {
         if (lane == 0) record_status(args.status, kStatusTimeout, 2);
         break;
       }
-      // this row's 2 x 96 packed bytes: chunk j of tile t at t*12288 + (j*128 + row)*16
-      const uint4* src = reinterpret_cast<const uint4*>(w_ring + s * Cfg::kWStageBytes) + row;
-      uint32_t w[4][12];
+      tc_fence_after();                           // the MMAs that read slot a are done
+      // this row's packed bytes: tile t, chunk j at t*12288 + (j*128 + row)*16
+      const uint4* src = reinterpret_cast<const uint4*>(w_ring + st.idx * Cfg::kWStageBytes) + row;
+      const uint32_t col = tmem + lane_base + Cfg::kACol0 + as.idx * Cfg::kACols;
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
+        uint32_t w[24];
 #pragma unroll
         for (int j = 0; j < 6; ++j) {
           const uint4 v = src[t * (kWTileBytes / 16) + j * 128];
-          uint32_t* d = &w[2 * t + j / 3][4 * (j % 3)];
-          d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+          w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
         }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctrl->empty[s]);
-      tc_fence_after();                     // A slot s is free: see GemmCfg
-      const uint32_t col = tmem + lane_base + Cfg::kACol0 + s * Cfg::kACols;
+        if (t == 1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctrl->empty[st.idx]);
+        }
+        uint32_t out[32];
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        uint32_t out[16];
-        unpack48(w[h], out);
-        tmem_st16(col + 16 * h, out);
+        for (int b = 0; b < 8; ++b) unpack_block(w[3 * b], w[3 * b + 1], w[3 * b + 2], &out[4 * b]);
+        tmem_st32(col + 32 * t, out);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctrl->a_full[s]);
+      if (lane == 0) mbar_arrive(&ctrl->a_full[as.idx]);
+      st.next();
+      as.next();
     }
     if (q == 0 && lane == 0) FLEXQ_ROLE_DONE(2, nst);
   } else {
     // ------------------------------------------------------ epilogue -----
+    constexpr int CH = Cfg::kLdChunk;
     const int e = warp - 6;
     const int q = warp & 3;
     const int c = e >> 2;
@@ -480,8 +495,8 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const int m_base = mt * T + col0;
     FLEXQ_ROLE_CLOCK;
+    RingPos<NB> pb;
     for (int lg = 0; lg < ngroups; ++lg) {
-      const int b = lg % Cfg::kPBufs;
       const int g = g0 + lg;
       const int gi = lg & 7;
       const int sc_slot = (lg >> 3) % Cfg::kScSlots;
@@ -495,7 +510,6 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
           }
           // this warp's tokens of the octet, FP16 -> FP32, into its own buffer
           const __half* sa_h = reinterpret_cast<const __half*>(sc);
-          __syncwarp();
 #pragma unroll
           for (int idx = lane; idx < 8 * Cfg::kCols; idx += 32) {
             const int gg = idx / Cfg::kCols, j = idx - gg * Cfg::kCols;
@@ -507,27 +521,22 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         swn = __half2float(sw_h[gi * kTileRows + row]) * 0.25f;   // TMEM holds 4 * code
       }
       const float* sa_w = ctrl->sa[e][gi];
-      if (!FLEXQ_WAIT(warp_wait(&ctrl->p_full[b], (lg / Cfg::kPBufs) & 1, lim))) {
+      if (!FLEXQ_WAIT(warp_wait(&ctrl->p_full[pb.idx], pb.phase, lim))) {
         if (lane == 0) record_status(args.status, kStatusTimeout, 4);
         break;
       }
       tc_fence_after();
       // drain the partials in chunks; the buffer is released right after the
       // last chunk has been read, before that chunk's arithmetic
-      constexpr int CH = Cfg::kLdChunk;
 #pragma unroll
       for (int ch = 0; ch < Cfg::kCols / CH; ++ch) {
         uint32_t pv[CH];
-#pragma unroll
-        for (int h = 0; h < CH / 16; ++h) {
-          uint32_t (&r)[16] = *reinterpret_cast<uint32_t(*)[16]>(&pv[16 * h]);
-          tmem_ld16(tmem + lane_base + Cfg::kPCol0 + b * T + col0 + ch * CH + 16 * h, r);
-        }
+        tmem_ld_cols<CH>(tmem + lane_base + Cfg::kPCol0 + pb.idx * T + col0 + ch * CH, pv);
         tmem_wait_ld();
         if (ch == Cfg::kCols / CH - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&ctrl->p_empty[b]);
+          if (lane == 0) mbar_arrive(&ctrl->p_empty[pb.idx]);
         }
         if (PARTIALS) {
 #pragma unroll
@@ -560,6 +569,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->s_empty[sc_slot]);
       }
+      pb.next();
     }
     if (e == 0 && lane == 0) FLEXQ_ROLE_DONE(3, ngroups);
   }

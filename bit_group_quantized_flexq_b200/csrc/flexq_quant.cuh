@@ -106,12 +106,33 @@ __global__ void __launch_bounds__(256) weight_scale_kernel(
 }
 
 // --------------------------------------------------------------------------
+// Device form of the packed weights.  The codes of 16 consecutive k of a row
+// form one 12-byte block of three little-endian 32-bit words w0, w1, w2:
+// byte t of word i holds the 6-bit code 4i+t in its bits [7:2] and bits
+// [2i+1:2i] of code 12+t in its bits [1:0].  Twelve codes are thus already
+// in place as int8 values code*4 (w & 0xFCFCFCFC), and the last four are
+// gathered from the three 2-bit pieces.  Rows are tiled as 128 rows x 128
+// codes (12288 bytes): tile (nt, kb) at (nt*(K/128) + kb) * 12288, and the
+// 96 bytes of row r inside it as six 16-byte chunks, chunk j at
+// (j*128 + r) * 16.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void pack_block(const uint32_t (&u)[16], uint32_t& w0,
+                                           uint32_t& w1, uint32_t& w2) {
+  uint32_t w[3] = {0u, 0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      w[i] |= (u[4 * i + t] << (8 * t + 2)) | (((u[12 + t] >> (2 * i)) & 3u) << (8 * t));
+  w0 = w[0];
+  w1 = w[1];
+  w2 = w[2];
+}
+
+// --------------------------------------------------------------------------
 // Weight quantization, pass 2: one thread per (row n, 64-code half of a
-// 128-code K-block).  It quantizes 64 values, packs them canonically into 48
-// bytes (four 6-bit codes per 24-bit little-endian word) and stores the three
-// 16-byte chunks at their device-form positions:
-//   tile (n/128, kb) at ((n/128)*(K/128) + kb) * 12288,
-//   chunk j of row r inside the tile at (j*128 + r) * 16.
+// 128-code K-block).  It quantizes 64 values into four 16-code blocks (48
+// bytes) and stores them as three 16-byte chunks at their tile positions.
 // --------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) weight_pack_kernel(
     const __half* __restrict__ W, const __half* __restrict__ Ws,
@@ -127,31 +148,22 @@ __global__ void __launch_bounds__(256) weight_pack_kernel(
   const uint4* p = reinterpret_cast<const uint4*>(W + static_cast<long long>(n) * K + k0);
   uint32_t word[12];
 #pragma unroll
-  for (int i = 0; i < 12; ++i) word[i] = 0;
+  for (int blk = 0; blk < 4; ++blk) {          // 16 codes = two 16-byte loads
+    uint32_t u[16];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {               // 8 values per 16-byte load
-    uint4 raw = __ldg(p + c);
-    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
-    const int kk = k0 + c * 8;
-    const float s = __half2float(Ws[static_cast<long long>(kk / gs) * N + n]);
-    uint32_t u[8];
+    for (int c = 0; c < 2; ++c) {
+      uint4 raw = __ldg(p + 2 * blk + c);
+      const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+      const int kk = k0 + 16 * blk + 8 * c;
+      const float s = __half2float(Ws[static_cast<long long>(kk / gs) * N + n]);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(h2[i]);
-      u[2 * i] = static_cast<uint32_t>(quant_code(f.x, s, 31)) & 0x3Fu;
-      u[2 * i + 1] = static_cast<uint32_t>(quant_code(f.y, s, 31)) & 0x3Fu;
-    }
-    // two quads -> two 24-bit words -> bytes 6c .. 6c+5 of the 48-byte run
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const uint32_t w24 = u[4 * q] | (u[4 * q + 1] << 6) | (u[4 * q + 2] << 12) |
-                           (u[4 * q + 3] << 18);
-#pragma unroll
-      for (int b = 0; b < 3; ++b) {
-        const int pos = 6 * c + 3 * q + b;    // byte position, compile time
-        word[pos >> 2] |= ((w24 >> (8 * b)) & 0xFFu) << (8 * (pos & 3));
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h2[i]);
+        u[8 * c + 2 * i] = static_cast<uint32_t>(quant_code(f.x, s, 31)) & 0x3Fu;
+        u[8 * c + 2 * i + 1] = static_cast<uint32_t>(quant_code(f.y, s, 31)) & 0x3Fu;
       }
     }
+    pack_block(u, word[3 * blk], word[3 * blk + 1], word[3 * blk + 2]);
   }
   const int nt = n >> 7, r = n & 127;
   uint8_t* tile = Wp + (static_cast<long long>(nt) * KB + kb) * 12288;
