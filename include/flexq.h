@@ -77,14 +77,16 @@ size_t flexq_weight_packed_bytes(int N, int K, int group_size);
  *
  *   W_fp16        [N, K] FP16, finite values.
  *   Wq_packed     out, flexq_weight_packed_bytes(N, K, gs) bytes: the device
- *                 form of the 6-bit codes.  Canonical packing: codes c0..c3 at
- *                 k = 4j..4j+3 of a row give the 24-bit little-endian word
- *                 (c0&63) | (c1&63)<<6 | (c2&63)<<12 | (c3&63)<<18.  Device
- *                 form: tiles of 128 rows x 128 codes (12288 bytes), tile
- *                 (nt, kb) at byte offset (nt*(K/128) + kb)*12288; inside a
- *                 tile, byte b of 16-byte chunk j (0..5) of row r holds
- *                 canonical byte kb*96 + 16*j + b of row nt*128 + r and sits
- *                 at offset (j*128 + r)*16 + b.
+ *                 form of the 6-bit codes, four codes per three bytes.  Each
+ *                 row is cut into blocks of 16 consecutive codes c0..c15
+ *                 (u_j = c_j & 63); a block is three little-endian 32-bit
+ *                 words w0, w1, w2 in which byte t of word i holds u_{4i+t}
+ *                 in its bits [7:2] and bits [2i+1:2i] of u_{12+t} in its
+ *                 bits [1:0].  The row's 96 bytes of codes kb*128 ..
+ *                 kb*128+127 (eight blocks) are cut into six 16-byte chunks;
+ *                 tile (nt, kb) (rows nt*128 .. nt*128+127) is 12288
+ *                 contiguous bytes at offset (nt*(K/128) + kb)*12288, and
+ *                 chunk j of row r sits at offset (j*128 + r)*16 inside it.
  *   W_scales_fp16 out, N*G FP16 values stored group-major: the scale of row
  *                 n, group g is element g*N + n.  s = fp16_rne(absmax / 31)
  *                 with absmax/31 computed as an IEEE FP32 division.
