@@ -248,13 +248,23 @@ int launch_gemm_t(DeviceState* st, const CUtensorMap& map, const CUtensorMap& ma
   cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes_for<T>(a.split));
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(a.split);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  // programmatic stream serialization: the kernel may start while the
+  // previous kernel of the stream finishes (it prefetches its weights, then
+  // waits for that kernel before reading activations)
+  cudaLaunchAttribute attr[2];
+  int nattr = 0;
+  attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[nattr].val.programmaticStreamSerializationAllowed = 1;
+  ++nattr;
+  if (a.split > 1) {
+    attr[nattr].id = cudaLaunchAttributeClusterDimension;
+    attr[nattr].val.clusterDim.x = static_cast<unsigned>(a.split);
+    attr[nattr].val.clusterDim.y = 1;
+    attr[nattr].val.clusterDim.z = 1;
+    ++nattr;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = a.split > 1 ? 1 : 0;
+  cfg.numAttrs = nattr;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map, map_sa, map_sw, a);
   if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
   return FLEXQ_OK;
@@ -377,13 +387,22 @@ int flexq_quantize_act(int M, int K, int group_size, int bits, const void* X_fp1
   __half* xs = static_cast<__half*>(X_scales_fp16);
   const int cpr = K / 8;
   const int ld = act_scales_ld(M);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   switch (group_size) {
-    case 32: flexq::quant_act_kernel<32><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, ld, qmax); break;
-    case 64: flexq::quant_act_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, ld, qmax); break;
-    case 128: flexq::quant_act_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, ld, qmax); break;
-    default: flexq::quant_act_kernel<256><<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, q, xs, chunks, cpr, ld, qmax); break;
+    case 32: e = cudaLaunchKernelEx(&cfg, flexq::quant_act_kernel<32>, x, q, xs, chunks, cpr, ld, qmax); break;
+    case 64: e = cudaLaunchKernelEx(&cfg, flexq::quant_act_kernel<64>, x, q, xs, chunks, cpr, ld, qmax); break;
+    case 128: e = cudaLaunchKernelEx(&cfg, flexq::quant_act_kernel<128>, x, q, xs, chunks, cpr, ld, qmax); break;
+    default: e = cudaLaunchKernelEx(&cfg, flexq::quant_act_kernel<256>, x, q, xs, chunks, cpr, ld, qmax); break;
   }
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "quant_act_kernel launch");
   return ok();
 }

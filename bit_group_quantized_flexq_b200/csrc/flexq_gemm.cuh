@@ -246,6 +246,9 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   const int lane = threadIdx.x & 31;
   const uint64_t lim = args.wait_limit_ns;
   FLEXQ_CTA_TIME(0);
+  // the next kernel of the stream may start its own prologue now; it waits
+  // for this grid before it reads anything this grid writes
+  if (threadIdx.x == 0) grid_launch_dependents();
 
   const int ks = blockIdx.x;            // K split index == rank in cluster
   const int nt = blockIdx.y;            // weight tile
@@ -308,6 +311,18 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       const int n_oct = PARTIALS ? 0 : (ngroups + 7) / 8;
       int next_oct = 0;
       bool ok = true;
+      // The packed weights are read-only inputs: the first ring's worth is
+      // requested before waiting for the kernels this one depends on (whose
+      // outputs may be this kernel's activations and their scales).
+      const int n_pre = nst < STAGES ? nst : STAGES;
+      for (int i = 0; i < n_pre; ++i) {
+        if (args.stall && i == 0) continue;
+        mbar_arrive_expect_tx(&ctrl->full[i], Cfg::kStageBytes);
+        bulk_load(w_ring + i * Cfg::kWStageBytes,
+                  args.wp + (static_cast<size_t>(nt) * KB + kb0 + 2 * i) * kWTileBytes,
+                  Cfg::kWStageBytes, &ctrl->full[i]);
+      }
+      grid_wait_dependencies();
       for (int i = 0; i < nst && ok; ++i) {
         // scales: issue octet o at the first stage that touches group 8*o
         const int lg_first = (i * Cfg::kKStage) >> gs_log2;
@@ -338,13 +353,15 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         if (args.stall && i == 0) continue;
         const int kb = kb0 + 2 * i;
         uint8_t* xs = xs_ring + s * Cfg::kXsBytes;
-        mbar_arrive_expect_tx(&ctrl->full[s], Cfg::kStageBytes);
+        if (i >= n_pre) {
+          mbar_arrive_expect_tx(&ctrl->full[s], Cfg::kStageBytes);
+          // tiles (nt, kb) and (nt, kb + 1) are adjacent in the device form
+          bulk_load(w_ring + s * Cfg::kWStageBytes,
+                    args.wp + (static_cast<size_t>(nt) * KB + kb) * kWTileBytes,
+                    Cfg::kWStageBytes, &ctrl->full[s]);
+        }
         tma_load_2d(xs, &tmap_x, &ctrl->full[s], kb * kKBlock, mt * T);
         tma_load_2d(xs + Cfg::kXsHalf, &tmap_x, &ctrl->full[s], (kb + 1) * kKBlock, mt * T);
-        // tiles (nt, kb) and (nt, kb + 1) are adjacent in the device form
-        bulk_load(w_ring + s * Cfg::kWStageBytes,
-                  args.wp + (static_cast<size_t>(nt) * KB + kb) * kWTileBytes,
-                  Cfg::kWStageBytes, &ctrl->full[s]);
         issued |= 1u << s;
         parity = (parity & ~(1u << s)) | (static_cast<uint32_t>((i / STAGES) & 1) << s);
       }

@@ -17,6 +17,18 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// --------------------------------------------- programmatic dependent launch
+// Lets the next kernel of the stream (launched with programmatic stream
+// serialization) start once every CTA of this grid has issued it.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Waits until the grids this one depends on have completed and their memory
+// operations are visible (returns at once when launched without dependency).
+__device__ __forceinline__ void grid_wait_dependencies() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------- mbarrier ----
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),

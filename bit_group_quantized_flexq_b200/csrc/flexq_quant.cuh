@@ -14,6 +14,8 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#include "flexq_ptx.cuh"
+
 namespace flexq {
 
 // Scale of a group from its absolute maximum.
@@ -38,6 +40,10 @@ __global__ void __launch_bounds__(256) quant_act_kernel(
     long long chunks, int chunks_per_row, int ld_scales, int qmax) {
   constexpr int LANES = GS / 8;            // lanes per group
   static_assert(LANES >= 4 && LANES <= 32, "group size 32..256");
+  // X may be the output of the previous kernel of the stream, and Xq / Xs
+  // may still be read by it: wait for it before touching either
+  grid_launch_dependents();
+  grid_wait_dependencies();
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   const long long first = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   // every lane of a warp runs the same number of iterations (the stride and
