@@ -133,6 +133,14 @@ int max_split_for(int T) {
   }
 }
 
+// Split-K workspace: kCounterBytes of arrival counters (one per output tile,
+// zero between calls) at a fixed place, then per output tile `split` FP32
+// partial tiles of T x 128.  The counters never move, so calls of different
+// shapes can share one workspace without their partial tiles landing on
+// another shape's counters.
+constexpr size_t kCounterBytes = 4096;
+constexpr long long kMaxSplitTiles = kCounterBytes / sizeof(unsigned);
+
 struct Plan {
   int T;
   int split;
@@ -156,7 +164,7 @@ Plan make_plan(int M, int N, int K, int gs, int sms, bool partials) {
     if (p.split > max_split_for(p.T)) p.split = max_split_for(p.T);
   }
   if (fS >= 1 && fS <= max_split_for(p.T) && fS <= units) p.split = fS;
-  if (partials) p.split = 1;
+  if (partials || tiles > kMaxSplitTiles) p.split = 1;
   p.ctas = static_cast<long long>(p.split) * (N / 128) * ((M + p.T - 1) / p.T);
   return p;
 }
@@ -213,17 +221,19 @@ int act_scales_ld(int M) { return (M + 7) / 8 * 8; }
 
 // --------------------------------------------------------------- launches --
 template <int T>
-int ctrl_offset_for(int split) {
-  using Cfg = flexq::GemmCfg<T>;
-  int stage = Cfg::kMainBytes;
-  int red = (split - 1) * 128 * T * 4;
-  int off = stage > red ? stage : red;
-  return (off + 15) & ~15;
+int ctrl_offset_for() {
+  return (flexq::GemmCfg<T>::kMainBytes + 15) & ~15;
 }
 
 template <int T>
-int smem_bytes_for(int split) {
-  return 1024 + ctrl_offset_for<T>(split) + static_cast<int>(sizeof(flexq::GemmCtrl<T>));
+int smem_bytes_for() {
+  return 1024 + ctrl_offset_for<T>() + static_cast<int>(sizeof(flexq::GemmCtrl<T>));
+}
+
+size_t workspace_bytes_for(const Plan& p, int M, int N) {
+  if (p.split <= 1) return 0;
+  const size_t tiles = static_cast<size_t>(N / 128) * ((M + p.T - 1) / p.T);
+  return kCounterBytes + tiles * static_cast<size_t>(p.split) * p.T * 128 * sizeof(float);
 }
 
 template <int T, bool PARTIALS>
@@ -236,42 +246,34 @@ int launch_gemm_t(DeviceState* st, const CUtensorMap& map, const CUtensorMap& ma
     std::lock_guard<std::mutex> lock(g_dev_mutex);
     if (!(st->attr_mask & bit)) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           smem_bytes_for<T>(Cfg::kMaxSplit));
+                                           smem_bytes_for<T>());
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
       st->attr_mask |= bit;
     }
   }
-  a.ctrl_offset = ctrl_offset_for<T>(a.split);
+  a.ctrl_offset = ctrl_offset_for<T>();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(a.split), static_cast<unsigned>(a.N / 128),
                      static_cast<unsigned>((a.M + T - 1) / T));
   cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes_for<T>(a.split));
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes_for<T>());
   cfg.stream = stream;
   // programmatic stream serialization: the kernel may start while the
   // previous kernel of the stream finishes (it prefetches its weights, then
   // waits for that kernel before reading activations)
-  cudaLaunchAttribute attr[2];
-  int nattr = 0;
-  attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[nattr].val.programmaticStreamSerializationAllowed = 1;
-  ++nattr;
-  if (a.split > 1) {
-    attr[nattr].id = cudaLaunchAttributeClusterDimension;
-    attr[nattr].val.clusterDim.x = static_cast<unsigned>(a.split);
-    attr[nattr].val.clusterDim.y = 1;
-    attr[nattr].val.clusterDim.z = 1;
-    ++nattr;
-  }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = nattr;
+  cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map, map_sa, map_sw, a);
   if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
   return FLEXQ_OK;
 }
 
 int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, const void* Wp,
-                const void* Ws, void* Y, int32_t* P, bool partials, void* stream) {
+                const void* Ws, void* Y, int32_t* P, bool partials, void* workspace,
+                size_t workspace_bytes, void* stream) {
   int rc = check_gemm_shape(M, N, K, gs);
   if (rc) return rc;
   if (M == 0) return ok();               // empty batch: nothing to read or write
@@ -286,7 +288,18 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
   }
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
-  const Plan plan = make_plan(M, N, K, gs, st->sms, partials);
+  Plan plan = make_plan(M, N, K, gs, st->sms, partials);
+  const size_t need = workspace_bytes_for(plan, M, N);
+  if (need > 0) {
+    if (workspace == nullptr && workspace_bytes == 0) {
+      plan.split = 1;                      // no workspace: no K split
+    } else if (workspace == nullptr || workspace_bytes < need) {
+      return fail(FLEXQ_ERR_INVALID_ARG, "workspace of %zu bytes at %p, the plan needs %zu",
+                  workspace_bytes, workspace, need);
+    } else if (!aligned16(workspace)) {
+      return fail(FLEXQ_ERR_MISALIGNED, "workspace is not 16-byte aligned");
+    }
+  }
   CUtensorMap map, map_sa, map_sw;
   if ((rc = encode_x_map(&map, Xq, M, K, plan.T))) return rc;
   memset(&map_sa, 0, sizeof(map_sa));
@@ -300,6 +313,10 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
   a.wp = static_cast<const uint8_t*>(Wp);
   a.y = static_cast<__half*>(Y);
   a.p = P;
+  if (plan.split > 1) {
+    a.ws_cnt = static_cast<unsigned int*>(workspace);
+    a.ws_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kCounterBytes);
+  }
   a.status = st->status;
   a.wait_limit_ns = g_wait_limit_ns.load();
   a.M = M; a.N = N; a.K = K; a.gs = gs; a.split = plan.split;
@@ -407,22 +424,31 @@ int flexq_quantize_act(int M, int K, int group_size, int bits, const void* X_fp1
   return ok();
 }
 
+size_t flexq_gemm_workspace_bytes(int M, int N, int K, int group_size) {
+  if (M <= 0 || N <= 0 || K <= 0 || N % 128 || K % 256 || !valid_gs(group_size) || K % group_size)
+    return 0;
+  const Plan p = make_plan(M, N, K, group_size, sm_count_or_default(), false);
+  return workspace_bytes_for(p, M, N);
+}
+
 int flexq_gemm_w6a6(int M, int N, int K, int group_size, const int8_t* Xq, const void* X_scales,
-                    const void* Wq_packed, const void* W_scales, void* Y_fp16, void* stream) {
+                    const void* Wq_packed, const void* W_scales, void* Y_fp16, void* workspace,
+                    size_t workspace_bytes, void* stream) {
   return gemm_common(M, N, K, group_size, Xq, X_scales, Wq_packed, W_scales, Y_fp16, nullptr,
-                     false, stream);
+                     false, workspace, workspace_bytes, stream);
 }
 
 int flexq_gemm_w6a8(int M, int N, int K, int group_size, const int8_t* Xq, const void* X_scales,
-                    const void* Wq_packed, const void* W_scales, void* Y_fp16, void* stream) {
+                    const void* Wq_packed, const void* W_scales, void* Y_fp16, void* workspace,
+                    size_t workspace_bytes, void* stream) {
   return gemm_common(M, N, K, group_size, Xq, X_scales, Wq_packed, W_scales, Y_fp16, nullptr,
-                     false, stream);
+                     false, workspace, workspace_bytes, stream);
 }
 
 int flexq_debug_group_partials(int M, int N, int K, int group_size, const int8_t* Xq,
                                const void* Wq_packed, int32_t* P, void* stream) {
   return gemm_common(M, N, K, group_size, Xq, nullptr, Wq_packed, nullptr, nullptr, P, true,
-                     stream);
+                     nullptr, 0, stream);
 }
 
 int flexq_gemm_plan(int M, int N, int K, int group_size, int* tile_tokens, int* k_split,

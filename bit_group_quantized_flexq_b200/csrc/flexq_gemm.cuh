@@ -11,8 +11,9 @@
 //
 // Orientation ("swap AB"): the MMA's M side is 128 weight rows, its N side
 // is T tokens.  Per CTA: one 128-row weight tile, one T-token tile and a
-// contiguous, group-aligned range of K (a cluster of `split` CTAs shares the
-// output tile and reduces through distributed shared memory).
+// contiguous, group-aligned range of K.  With a K split, the `split` CTAs of
+// an output tile write FP32 partial tiles to a workspace and the last one to
+// finish adds them in split order (see the teardown).
 //
 // The pipeline advances in stages of 256 codes of K (two 128 x 128 weight
 // tiles).
@@ -33,7 +34,8 @@
 //   warps 6..   epilogue: per group, load the int32 partials from TMEM,
 //               release the buffer, and accumulate
 //               acc += float(P) * (sw[n,g]/4 * sa[m,g]) in FP32 registers;
-//               at the end store FP16 (or reduce across the cluster first).
+//               at the end store FP16 (or hand the partial tile to the
+//               split-K reduction).
 #pragma once
 
 #include <cuda.h>
@@ -54,6 +56,8 @@ struct GemmArgs {
   const uint8_t* wp;       // packed weights, device form
   __half* y;               // [M, N] output (GEMM mode)
   int32_t* p;              // [G, M, N] partials (debug mode)
+  float* ws_part;          // split-K partial tiles [tiles][split][T][128] (split > 1)
+  unsigned int* ws_cnt;    // split-K arrival counters [tiles], zero between calls
   unsigned int* status;    // device status word [4]
   unsigned long long wait_limit_ns;
   int M, N, K, gs, split;
@@ -112,7 +116,7 @@ struct GemmCtrl {
   uint64_t s_empty[GemmCfg<T>::kScSlots];
   uint64_t done;
   uint32_t tmem_base;
-  uint32_t pad;
+  uint32_t is_last;        // split-K: this CTA reduces the output tile
   // per epilogue warp: its tokens' activation scales of the current octet, FP32
   alignas(16) float sa[GemmCfg<T>::kEpiWarps][8][GemmCfg<T>::kCols];
 };
@@ -132,7 +136,7 @@ struct RingPos {
 
 // Optional pipeline trace (compile with -DFLEXQ_TRACE).  Every CTA records
 // %globaltimer at entry (0), after set-up (1), after its roles' loops (2), at
-// exit (3), after the TMEM release (5), after the first cluster barrier (6)
+// exit (3), after the TMEM release (5), after the split-K partial store (6)
 // and before the output store (7), with its SM id in slot 4.  CTA 0 and the
 // CTA in the middle of the grid also record, per role (producer, MMA, unpack
 // warp of lane quarter 0, first epilogue warp), the cycles spent in the role
@@ -239,7 +243,6 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   uint8_t* xs_ring = base;                                  // STAGES * kXsBytes
   uint8_t* w_ring = base + STAGES * Cfg::kXsBytes;          // STAGES * 24576
   uint8_t* sc_ring = w_ring + STAGES * Cfg::kWStageBytes;   // kScSlots slots
-  float* red = reinterpret_cast<float*>(base);              // cluster reduction
   GemmCtrl<T>* ctrl = reinterpret_cast<GemmCtrl<T>*>(base + args.ctrl_offset);
 
   const int warp = threadIdx.x >> 5;
@@ -250,7 +253,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   // for this grid before it reads anything this grid writes
   if (threadIdx.x == 0) grid_launch_dependents();
 
-  const int ks = blockIdx.x;            // K split index == rank in cluster
+  const int ks = blockIdx.x;            // K split index
   const int nt = blockIdx.y;            // weight tile
   const int mt = blockIdx.z;            // token tile
   const int M = args.M, N = args.N, K = args.K, gs = args.gs, S = args.split;
@@ -610,31 +613,50 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   const int row = (warp & 3) * 32 + lane;
   const int col0 = (e >> 2) * Cfg::kCols;
   if (S > 1) {
-    // split-K: ranks 1..S-1 add their partial tiles into rank 0's shared
-    // memory (the stage ring is idle now), in a fixed order
-    cluster_sync_all();
-    FLEXQ_CTA_TIME(6);
-    if (is_epi && ks != 0) {
-      const uint32_t remote = map_to_rank(smem_u32(red), 0);
+    // split-K: every CTA writes its FP32 partial tile to the workspace; the
+    // last CTA of the output tile to arrive adds the `split` partials in
+    // split order (the same order whichever CTA arrives last, so the result
+    // is deterministic), writes the FP16 output and resets the counter.
+    const size_t tile = static_cast<size_t>(mt) * gridDim.y + nt;
+    float* part = args.ws_part + tile * static_cast<size_t>(S) * T * kTileRows;
+    if (is_epi) {
 #pragma unroll
-      for (int j = 0; j < Cfg::kCols; ++j) {
-        const uint32_t off = static_cast<uint32_t>(((ks - 1) * T + col0 + j) * kTileRows + row);
-        st_cluster_f32(remote + off * 4u, (j & 1) ? acc[j / 2].y : acc[j / 2].x);
-      }
+      for (int j = 0; j < Cfg::kCols; ++j)
+        part[(static_cast<size_t>(ks) * T + col0 + j) * kTileRows + row] =
+            (j & 1) ? acc[j / 2].y : acc[j / 2].x;
     }
-    cluster_sync_all();
-    if (ks != 0) {
+    __threadfence();
+    __syncthreads();
+    FLEXQ_CTA_TIME(6);
+    if (threadIdx.x == 0) {
+      const unsigned old = atomicAdd(&args.ws_cnt[tile], 1u);
+      const bool last = old == static_cast<unsigned>(S - 1);
+      if (last) args.ws_cnt[tile] = 0u;
+      ctrl->is_last = last ? 1u : 0u;
+    }
+    __syncthreads();
+    if (!ctrl->is_last) {
       FLEXQ_CTA_TIME(3);
       return;
     }
+    __threadfence();
     if (is_epi) {
-      for (int r = 1; r < S; ++r) {
+      float2 sum[Cfg::kCols / 2];
+#pragma unroll
+      for (int j = 0; j < Cfg::kCols / 2; ++j) sum[j] = make_float2(0.0f, 0.0f);
+      for (int r = 0; r < S; ++r) {
+        const float* pr = part + (static_cast<size_t>(r) * T + col0) * kTileRows + row;
 #pragma unroll
         for (int j = 0; j < Cfg::kCols; j += 2) {
-          acc[j / 2].x += red[((r - 1) * T + col0 + j) * kTileRows + row];
-          acc[j / 2].y += red[((r - 1) * T + col0 + j + 1) * kTileRows + row];
+          // this CTA's own partial from registers, the others from L2
+          const float x0 = (r == ks) ? acc[j / 2].x : __ldcg(pr + j * kTileRows);
+          const float x1 = (r == ks) ? acc[j / 2].y : __ldcg(pr + (j + 1) * kTileRows);
+          sum[j / 2].x += x0;
+          sum[j / 2].y += x1;
         }
       }
+#pragma unroll
+      for (int j = 0; j < Cfg::kCols / 2; ++j) acc[j] = sum[j];
     }
   }
   FLEXQ_CTA_TIME(7);

@@ -49,10 +49,13 @@ def lib():
                                               c_void_p, c_void_p]),
             "flexq_quantize_act": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p,
                                            c_void_p, c_void_p]),
+            "flexq_gemm_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
             "flexq_gemm_w6a6": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p,
-                                        c_void_p, c_void_p, c_void_p, c_void_p]),
+                                        c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                        c_void_p]),
             "flexq_gemm_w6a8": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p,
-                                        c_void_p, c_void_p, c_void_p, c_void_p]),
+                                        c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                        c_void_p]),
             "flexq_debug_group_partials": (c_int, [c_int, c_int, c_int, c_int, c_void_p,
                                                    c_void_p, c_void_p, c_void_p]),
             "flexq_gemm_plan": (c_int, [c_int, c_int, c_int, c_int,
@@ -153,8 +156,43 @@ def quantize_act(x, group_size, bits, out=None):
     return xq, xs
 
 
-def gemm(xq, xs, wp, ws, N, group_size, act_bits=6, out=None):
-    """Y [M, N] FP16 = dequant(xq, xs) . dequant(wp, ws)^T (W6A6 or W6A8)."""
+def gemm_workspace_bytes(M, N, K, group_size):
+    return int(lib().flexq_gemm_workspace_bytes(M, N, K, group_size))
+
+
+# zero-filled split-K workspaces, one growing buffer per device; superseded
+# buffers stay alive because captured CUDA graphs may still point at them
+_workspaces = {}
+_retired = []
+
+
+def workspace(device, nbytes):
+    """A zero-filled device workspace of at least `nbytes` bytes on `device`
+    (shared by every call on that device that does not pass its own)."""
+    dev = torch.device(device)
+    key = (dev.type, dev.index if dev.index is not None else torch.cuda.current_device())
+    cur = _workspaces.get(key)
+    if cur is None or cur.numel() < nbytes:
+        if cur is not None:
+            _retired.append(cur)
+        cur = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=dev)
+        _workspaces[key] = cur
+    return cur
+
+
+def reset_workspaces():
+    """Zero every workspace handed out by `workspace` (after a device-side
+    timeout left split-K counters behind)."""
+    for t in list(_workspaces.values()) + _retired:
+        t.zero_()
+
+
+def gemm(xq, xs, wp, ws, N, group_size, act_bits=6, out=None, workspace_buf=None):
+    """Y [M, N] FP16 = dequant(xq, xs) . dequant(wp, ws)^T (W6A6 or W6A8).
+
+    workspace_buf: a zero-filled uint8 device tensor of at least
+    gemm_workspace_bytes(M, N, K, gs) bytes; by default a per-device shared
+    one.  Pass an empty tensor to run without a K split."""
     _need(xq, "xq", torch.int8)
     M, K = xq.shape
     _need(xs, "xs", torch.float16, (K // group_size, act_scales_ld(M)))
@@ -163,8 +201,17 @@ def gemm(xq, xs, wp, ws, N, group_size, act_bits=6, out=None):
     if out is None:
         out = torch.empty(M, N, dtype=torch.float16, device=xq.device)
     _need(out, "out", torch.float16, (M, N))
+    if workspace_buf is None:
+        need = gemm_workspace_bytes(M, N, K, group_size)
+        workspace_buf = workspace(xq.device, need) if need else None
+    if workspace_buf is None or workspace_buf.numel() == 0:
+        wsp, wsn = ctypes.c_void_p(0), 0
+    else:
+        _need(workspace_buf, "workspace", torch.uint8)
+        wsp, wsn = _ptr(workspace_buf), workspace_buf.numel()
     fn = {6: lib().flexq_gemm_w6a6, 8: lib().flexq_gemm_w6a8}[act_bits]
-    _check(fn(M, N, K, group_size, _ptr(xq), _ptr(xs), _ptr(wp), _ptr(ws), _ptr(out), _stream(xq)))
+    _check(fn(M, N, K, group_size, _ptr(xq), _ptr(xs), _ptr(wp), _ptr(ws), _ptr(out), wsp, wsn,
+              _stream(xq)))
     return out
 
 
@@ -211,4 +258,7 @@ def device_status(device=None):
     """Synchronizes the current stream and returns (status, message); clears it."""
     s = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
     st = lib().flexq_get_device_status(s)
-    return st, lib().flexq_last_error_message().decode()
+    msg = lib().flexq_last_error_message().decode()
+    if st == FLEXQ_ERR_DEVICE_TIMEOUT:
+        reset_workspaces()
+    return st, msg

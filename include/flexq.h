@@ -117,6 +117,16 @@ int flexq_quantize_act(int M, int K, int group_size, int bits,
                        void* stream);
 
 /*
+ * flexq_gemm_workspace_bytes -- device workspace the GEMM entry points need
+ * for a shape: 0 when the launch plan does not split K, otherwise 4096 bytes
+ * of arrival counters (one per output tile, always at the start, so calls of
+ * different shapes can share one workspace) followed by the FP32 partial
+ * tiles of the K split.  Pure host computation; 0 for unsupported shapes and
+ * M <= 0.  Plans with more than 1024 output tiles never split K.
+ */
+size_t flexq_gemm_workspace_bytes(int M, int N, int K, int group_size);
+
+/*
  * flexq_gemm_w6a6 / flexq_gemm_w6a8 -- Y = dequant(Xq) . dequant(Wq)^T.
  * Passage: the W6A6 / W6A8 GEMM whose integer products are summed per group
  * and recombined with the scales, dequantization fused into the GEMM (arXiv
@@ -128,10 +138,21 @@ int flexq_quantize_act(int M, int K, int group_size, int bits,
  *   W_scales         (group-major, g*N + n), as written by
  *                    flexq_quantize_weight.
  *   Y_fp16           out, [M, N] FP16.
+ *   workspace,       device scratch of flexq_gemm_workspace_bytes(M, N, K, gs)
+ *   workspace_bytes  bytes or more, owned by the caller, 16-byte aligned.  It
+ *                    must be zero-filled before its first use; every call
+ *                    that completes leaves it zero-filled again (re-zero it
+ *                    after a call that reported FLEXQ_ERR_DEVICE_TIMEOUT).
+ *                    Calls that share a workspace must not overlap on the
+ *                    GPU.  NULL with 0 bytes runs the GEMM without a K split
+ *                    (correct, slower at small M); a smaller non-zero size is
+ *                    FLEXQ_ERR_INVALID_ARG.
  * For each group g the integer partial P_g[m,n] = sum_{k in g} Xq[m,k]*Wq[n,k]
  * is formed exactly (int32), then Y[m,n] = fp16_rne(sum_g P_g[m,n] *
  * sa[m,g] * sw[n,g]) with the sum over groups accumulated in FP32 (per
  * output, |Y - Y_exact| <= 5e-4 * max|Y| on the benchmark distributions).
+ * A K split adds the FP32 partial sums of its ranges in a fixed order, so the
+ * output does not depend on the order in which the CTAs finish.
  * The two entry points run the same kernel: they differ only in the code
  * range the caller's activations are expected to use ([-31, 31] vs
  * [-127, 127]); neither checks the range, and any int8 activation code and
@@ -139,10 +160,12 @@ int flexq_quantize_act(int M, int K, int group_size, int bits,
  */
 int flexq_gemm_w6a6(int M, int N, int K, int group_size, const int8_t* Xq,
                     const void* X_scales, const void* Wq_packed,
-                    const void* W_scales, void* Y_fp16, void* stream);
+                    const void* W_scales, void* Y_fp16, void* workspace,
+                    size_t workspace_bytes, void* stream);
 int flexq_gemm_w6a8(int M, int N, int K, int group_size, const int8_t* Xq,
                     const void* X_scales, const void* Wq_packed,
-                    const void* W_scales, void* Y_fp16, void* stream);
+                    const void* W_scales, void* Y_fp16, void* workspace,
+                    size_t workspace_bytes, void* stream);
 
 /*
  * flexq_debug_group_partials -- exports the per-group int32 partials of the
@@ -154,10 +177,10 @@ int flexq_debug_group_partials(int M, int N, int K, int group_size,
                                int32_t* P, void* stream);
 
 /*
- * flexq_gemm_plan -- the launch the GEMM entry points would use for a shape:
- * tokens per tile (16, 32, 64 or 128), K-split factor (CTAs of one cluster
- * that share an output tile) and the number of CTAs.  Any output pointer may
- * be NULL.  Pure host computation.
+ * flexq_gemm_plan -- the launch the GEMM entry points would use for a shape
+ * given enough workspace: tokens per tile (16, 32, 64 or 128), K-split factor
+ * (CTAs that share an output tile, each over its own range of K) and the
+ * number of CTAs.  Any output pointer may be NULL.  Pure host computation.
  */
 int flexq_gemm_plan(int M, int N, int K, int group_size, int* tile_tokens,
                     int* k_split, int* ctas);

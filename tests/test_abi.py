@@ -72,12 +72,12 @@ def test_validation_before_any_launch(L):
     assert L.flexq_quantize_act(-1, 256, 128, 6, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
     # GEMM shape rules
     g = L.flexq_gemm_w6a6
-    assert g(4, 200, 256, 128, FAKE, FAKE, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
-    assert g(4, 256, 200, 128, FAKE, FAKE, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
-    assert g(4, 256, 384, 256, FAKE, FAKE, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
-    assert g(4, 256, 256, 128, FAKE, NULL, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
-    assert g(4, 256, 256, 128, FAKE, FAKE, FAKE, FAKE, MISALIGNED, NULL) == flexq.FLEXQ_ERR_MISALIGNED
-    assert L.flexq_gemm_w6a8(-3, 256, 256, 128, FAKE, FAKE, FAKE, FAKE, FAKE, NULL) == \
+    assert g(4, 200, 256, 128, FAKE, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
+    assert g(4, 256, 200, 128, FAKE, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
+    assert g(4, 256, 384, 256, FAKE, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
+    assert g(4, 256, 256, 128, FAKE, NULL, FAKE, FAKE, FAKE, NULL, 0, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert g(4, 256, 256, 128, FAKE, FAKE, FAKE, FAKE, MISALIGNED, NULL, 0, NULL) == flexq.FLEXQ_ERR_MISALIGNED
+    assert L.flexq_gemm_w6a8(-3, 256, 256, 128, FAKE, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == \
         flexq.FLEXQ_ERR_INVALID_ARG
     w = L.flexq_quantize_weight
     assert w(130, 256, 128, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
@@ -99,3 +99,15 @@ def test_plan_is_host_only_and_sane(L):
     t, s, c = flexq.plan(1, 4096, 256, 256)
     assert s == 1                     # one group: nothing to split
     assert flexq.plan(0, 256, 256, 128) == (0, 0, 0)
+
+
+def test_workspace_size_follows_the_plan(L):
+    # no K split: no workspace; a K split: FP32 partial tiles + one counter per tile
+    assert flexq.gemm_workspace_bytes(2048, 4096, 4096, 128) == 0 or flexq.plan(2048, 4096, 4096, 128)[1] > 1
+    for M, N, K in [(1, 4096, 4096), (16, 11008, 4096), (5, 384, 4096)]:
+        t, s, c = flexq.plan(M, N, K, 128)
+        tiles = (N // 128) * ((M + t - 1) // t)
+        want = 0 if s == 1 else 4096 + tiles * s * t * 128 * 4
+        assert flexq.gemm_workspace_bytes(M, N, K, 128) == want
+    assert flexq.gemm_workspace_bytes(0, 4096, 4096, 128) == 0
+    assert flexq.gemm_workspace_bytes(4, 200, 4096, 128) == 0

@@ -174,3 +174,48 @@ def test_stalled_pipeline_reports_timeout_and_context_survives():
     ref = orc.linear_layer(x.numpy(), w.numpy(), gs, 6)
     assert_within(np16(y), ref["y64"], TOL)
     assert flexq.device_status()[0] == flexq.FLEXQ_OK
+
+
+# ------------------------------------------------------ split-K workspace --
+def test_split_k_is_deterministic_and_leaves_the_workspace_zeroed():
+    M, N, K, gs, bits = 7, 384, 4096, 128, 6
+    x, w = _layer(M, N, K, gs, bits, seed=21)
+    wp, ws = flexq.quantize_weight(w.cuda(), gs)
+    xq, xs = flexq.quantize_act(x.cuda(), gs, bits)
+    flexq.force_plan(16, 8)
+    need = flexq.gemm_workspace_bytes(M, N, K, gs)
+    assert need > 0
+    buf = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    y1 = flexq.gemm(xq, xs, wp, ws, N, gs, bits, workspace_buf=buf).clone()
+    assert int(buf.count_nonzero()) > 0                      # partial tiles were written
+    counters = buf[:4096]                                    # fixed counter region
+    assert int(counters.count_nonzero()) == 0                # every counter reset
+    y2 = flexq.gemm(xq, xs, wp, ws, N, gs, bits, workspace_buf=buf)
+    assert torch.equal(y1, y2)                               # fixed reduction order
+    ref = orc.linear_layer(x.numpy(), w.numpy(), gs, bits)
+    assert_within(np16(y1), ref["y64"], TOL)
+
+
+def test_gemm_without_workspace_runs_without_a_k_split():
+    M, N, K, gs, bits = 3, 256, 2048, 64, 8
+    x, w = _layer(M, N, K, gs, bits, seed=22)
+    wp, ws = flexq.quantize_weight(w.cuda(), gs)
+    xq, xs = flexq.quantize_act(x.cuda(), gs, bits)
+    assert flexq.plan(M, N, K, gs)[1] > 1
+    y = flexq.gemm(xq, xs, wp, ws, N, gs, bits,
+                   workspace_buf=torch.empty(0, dtype=torch.uint8, device="cuda"))
+    ref = orc.linear_layer(x.numpy(), w.numpy(), gs, bits)
+    assert_within(np16(y), ref["y64"], TOL)
+
+
+def test_too_small_workspace_is_rejected():
+    M, N, K, gs = 2, 256, 2048, 128
+    x, w = _layer(M, N, K, gs, 6, seed=23)
+    wp, ws = flexq.quantize_weight(w.cuda(), gs)
+    xq, xs = flexq.quantize_act(x.cuda(), gs, 6)
+    need = flexq.gemm_workspace_bytes(M, N, K, gs)
+    assert need > 16
+    small = torch.zeros(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(flexq.FlexQError) as ei:
+        flexq.gemm(xq, xs, wp, ws, N, gs, 6, workspace_buf=small)
+    assert ei.value.status == flexq.FLEXQ_ERR_INVALID_ARG
