@@ -331,6 +331,36 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
   return rc ? rc : ok();
 }
 
+// --------------------------------------------------- static GEMM scratch --
+// Scratch of flexq_gemm_static_scratch, for callers that may not allocate
+// device memory: the same layout as a caller workspace (arrival counters,
+// then FP32 partial tiles), fixed at 16 MiB.  Every device that loads the
+// library holds it until the process exits.
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(16) << 20;
+static __device__ __align__(256) unsigned char g_flexq_static_scratch[kStaticScratchBytes];
+
+// Device address of the scratch on each device, looked up once per device
+// with that device current (host code may not use the symbol itself: in host
+// code it names a host-side stand-in, not device memory).
+void* g_static_scratch_ptr[kMaxDevices] = {};
+std::mutex g_static_scratch_mutex;
+
+int static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FLEXQ_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+  if (g_static_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_flexq_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    g_static_scratch_ptr[dev] = p;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return FLEXQ_OK;
+}
+
 }  // namespace
 
 // ===================================================================== ABI ==
@@ -443,6 +473,34 @@ int flexq_gemm_w6a8(int M, int N, int K, int group_size, const int8_t* Xq, const
                     size_t workspace_bytes, void* stream) {
   return gemm_common(M, N, K, group_size, Xq, X_scales, Wq_packed, W_scales, Y_fp16, nullptr,
                      false, workspace, workspace_bytes, stream);
+}
+
+int flexq_gemm_static_scratch(int M, int N, int K, int group_size, int act_bits,
+                              const int8_t* Xq, const void* X_scales, const void* Wq_packed,
+                              const void* W_scales, void* Y_fp16, void* stream) {
+  if (act_bits != 6 && act_bits != 8)
+    return fail(FLEXQ_ERR_INVALID_ARG, "act_bits=%d is not 6 or 8", act_bits);
+  int rc = check_gemm_shape(M, N, K, group_size);
+  if (rc) return rc;
+  if (M == 0) return ok();
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  const size_t need = workspace_bytes_for(make_plan(M, N, K, group_size, st->sms, false), M, N);
+  if (need > kStaticScratchBytes)
+    return fail(FLEXQ_ERR_UNSUPPORTED,
+                "this shape needs %zu bytes of split-K scratch, more than the %zu of the "
+                "static scratch; use flexq_gemm_w6a6/w6a8 with a workspace", need,
+                kStaticScratchBytes);
+  void* scratch = nullptr;
+  if ((rc = static_scratch(&scratch))) return rc;
+  if (need > 0) {
+    // the arrival counters must start at zero; earlier calls leave them zero
+    // unless one of them gave up on a wait, so clear them every time
+    cudaError_t e = cudaMemsetAsync(scratch, 0, kCounterBytes, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the static scratch counters");
+  }
+  return gemm_common(M, N, K, group_size, Xq, X_scales, Wq_packed, W_scales, Y_fp16, nullptr,
+                     false, scratch, kStaticScratchBytes, stream);
 }
 
 int flexq_debug_group_partials(int M, int N, int K, int group_size, const int8_t* Xq,

@@ -56,6 +56,9 @@ def lib():
             "flexq_gemm_w6a8": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p,
                                         c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                         c_void_p]),
+            "flexq_gemm_static_scratch": (c_int, [c_int, c_int, c_int, c_int, c_int, c_void_p,
+                                                  c_void_p, c_void_p, c_void_p, c_void_p,
+                                                  c_void_p]),
             "flexq_debug_group_partials": (c_int, [c_int, c_int, c_int, c_int, c_void_p,
                                                    c_void_p, c_void_p, c_void_p]),
             "flexq_gemm_plan": (c_int, [c_int, c_int, c_int, c_int,
@@ -212,6 +215,23 @@ def gemm(xq, xs, wp, ws, N, group_size, act_bits=6, out=None, workspace_buf=None
     fn = {6: lib().flexq_gemm_w6a6, 8: lib().flexq_gemm_w6a8}[act_bits]
     _check(fn(M, N, K, group_size, _ptr(xq), _ptr(xs), _ptr(wp), _ptr(ws), _ptr(out), wsp, wsn,
               _stream(xq)))
+    return out
+
+
+def gemm_static_scratch(xq, xs, wp, ws, N, group_size, act_bits=6, out=None):
+    """The GEMM through flexq_gemm_static_scratch: no workspace argument and
+    no device allocation by the library (the split-K scratch is a fixed array
+    in device memory shared by all such calls on a device)."""
+    _need(xq, "xq", torch.int8)
+    M, K = xq.shape
+    _need(xs, "xs", torch.float16, (K // group_size, act_scales_ld(M)))
+    _need(wp, "wp", torch.uint8, (weight_packed_bytes(N, K, group_size),))
+    _need(ws, "ws", torch.float16, (K // group_size, N))
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.float16, device=xq.device)
+    _need(out, "out", torch.float16, (M, N))
+    _check(lib().flexq_gemm_static_scratch(M, N, K, group_size, act_bits, _ptr(xq), _ptr(xs),
+                                           _ptr(wp), _ptr(ws), _ptr(out), _stream(xq)))
     return out
 
 

@@ -168,6 +168,31 @@ int flexq_gemm_w6a8(int M, int N, int K, int group_size, const int8_t* Xq,
                     size_t workspace_bytes, void* stream);
 
 /*
+ * flexq_gemm_static_scratch -- the GEMM of flexq_gemm_w6a6 (act_bits 6) or
+ * flexq_gemm_w6a8 (act_bits 8) for callers that cannot allocate device
+ * memory when they call it: an engine plugin whose enqueue step may not
+ * allocate, or a serving process that reserves all device memory for its own
+ * pool at start-up.  The paper has no counterpart; this is an interface
+ * convenience of this library.
+ *   Same arguments, layouts and results as flexq_gemm_w6a6/w6a8 without the
+ *   workspace: the split-K scratch is a 16 MiB array the library keeps in
+ *   each device's global memory for the life of the process.  The call
+ *   allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ *   Shapes whose plan needs more split-K scratch than 16 MiB are rejected
+ *   with FLEXQ_ERR_UNSUPPORTED (no plan the library picks by itself does).
+ *   The first call on a device looks up the scratch's device address; make
+ *   that first call before capturing a stream.  Each call first clears the
+ *   scratch's arrival counters on `stream` (a 4 KB memset), then launches.
+ *   All calls on a device share the one scratch, which keeps the last call's
+ *   partial tiles: two calls that overlap on the GPU (different streams, or
+ *   concurrently running graphs) race on it and give wrong results.
+ */
+int flexq_gemm_static_scratch(int M, int N, int K, int group_size, int act_bits,
+                              const int8_t* Xq, const void* X_scales,
+                              const void* Wq_packed, const void* W_scales,
+                              void* Y_fp16, void* stream);
+
+/*
  * flexq_debug_group_partials -- exports the per-group int32 partials of the
  * GEMM above, computed by the same kernel mainloop (test hook).
  *   P  out, int32 [G, M, N]: P[g][m][n] = sum_{k in g} Xq[m,k] * Wq[n,k].
