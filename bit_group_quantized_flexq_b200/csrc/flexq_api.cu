@@ -423,16 +423,37 @@ int flexq_quantize_act(int M, int K, int group_size, int bits, const void* X_fp1
   if (rc) return rc;
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
-  const long long chunks = static_cast<long long>(M) * K / 8;
-  long long blocks = (chunks + 255) / 256;
-  const long long cap = static_cast<long long>(st->sms) * 16;
-  if (blocks > cap) blocks = cap;
+  // Grid: whole rows per step (the thread count a multiple of the row length
+  // in 16-byte chunks, cpr = K/8), at most one resident wave; each thread
+  // keeps four loads in flight and strides over the remaining rows.
+  const int cpr = K / 8;
+  if (static_cast<long long>(M) * cpr >= (1ll << 31))
+    return fail(FLEXQ_ERR_UNSUPPORTED, "M*K/8 = %lld chunks exceeds 2^31", static_cast<long long>(M) * cpr);
+  int per_sm = 0;
+  cudaError_t oe = cudaSuccess;
+  switch (group_size) {
+    case 32: oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, flexq::quant_act_kernel<32>, 256, 0); break;
+    case 64: oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, flexq::quant_act_kernel<64>, 256, 0); break;
+    case 128: oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, flexq::quant_act_kernel<128>, 256, 0); break;
+    default: oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, flexq::quant_act_kernel<256>, 256, 0); break;
+  }
+  if (oe != cudaSuccess || per_sm < 1) per_sm = 4;
+  // blocks per group of whole rows: the smallest b with b*256 a multiple of cpr
+  long long g = cpr, h = 256;                 // gcd(cpr, 256)
+  while (h) { const long long r = g % h; g = h; h = r; }
+  const long long unit_blocks = cpr / g;       // blocks that hold whole rows
+  const long long unit_rows = unit_blocks * 256 / cpr;
+  long long units = static_cast<long long>(st->sms) * per_sm / unit_blocks;
+  if (units < 1) units = 1;
+  const long long need_units = (M + unit_rows - 1) / unit_rows;
+  if (units > need_units) units = need_units;
+  const long long blocks = units * unit_blocks;
+  const int rows_per_step = static_cast<int>(units * unit_rows);
   const int qmax = bits == 6 ? 31 : 127;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint4* x = static_cast<const uint4*>(X_fp16);
   uint2* q = reinterpret_cast<uint2*>(Xq);
   __half* xs = static_cast<__half*>(X_scales_fp16);
-  const int cpr = K / 8;
   const int ld = act_scales_ld(M);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
@@ -445,10 +466,10 @@ int flexq_quantize_act(int M, int K, int group_size, int bits, const void* X_fp1
   cfg.numAttrs = 1;
   cudaError_t e;
   switch (group_size) {
-    case 32: e = cudaLaunchKernelEx(&cfg, flexq::quant_act_kernel<32>, x, q, xs, chunks, cpr, ld, qmax); break;
-    case 64: e = cudaLaunchKernelEx(&cfg, flexq::quant_act_kernel<64>, x, q, xs, chunks, cpr, ld, qmax); break;
-    case 128: e = cudaLaunchKernelEx(&cfg, flexq::quant_act_kernel<128>, x, q, xs, chunks, cpr, ld, qmax); break;
-    default: e = cudaLaunchKernelEx(&cfg, flexq::quant_act_kernel<256>, x, q, xs, chunks, cpr, ld, qmax); break;
+    case 32: e = cudaLaunchKernelEx(&cfg, flexq::quant_act_kernel<32>, x, q, xs, M, cpr, rows_per_step, ld, qmax); break;
+    case 64: e = cudaLaunchKernelEx(&cfg, flexq::quant_act_kernel<64>, x, q, xs, M, cpr, rows_per_step, ld, qmax); break;
+    case 128: e = cudaLaunchKernelEx(&cfg, flexq::quant_act_kernel<128>, x, q, xs, M, cpr, rows_per_step, ld, qmax); break;
+    default: e = cudaLaunchKernelEx(&cfg, flexq::quant_act_kernel<256>, x, q, xs, M, cpr, rows_per_step, ld, qmax); break;
   }
   if (e != cudaSuccess) return cuda_fail(e, "quant_act_kernel launch");
   return ok();
@@ -501,6 +522,32 @@ int flexq_gemm_static_scratch(int M, int N, int K, int group_size, int act_bits,
   }
   return gemm_common(M, N, K, group_size, Xq, X_scales, Wq_packed, W_scales, Y_fp16, nullptr,
                      false, scratch, kStaticScratchBytes, stream);
+}
+
+int flexq_debug_check_quantizer(unsigned long long* mismatches, unsigned int* first_mismatch) {
+  if (!mismatches || !first_mismatch)
+    return fail(FLEXQ_ERR_INVALID_ARG, "mismatches and first_mismatch must not be NULL");
+  unsigned long long* d_count = nullptr;
+  unsigned* d_first = nullptr;
+  // test hook only: the library's product entry points never allocate
+  cudaError_t e = cudaMalloc(&d_count, sizeof(unsigned long long) + 4 * sizeof(unsigned));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc");
+  d_first = reinterpret_cast<unsigned*>(d_count + 1);
+  e = cudaMemset(d_count, 0, sizeof(unsigned long long) + 4 * sizeof(unsigned));
+  // every positive finite FP16 scale (0x0001 .. 0x7BFF), 1024 scales per launch
+  for (unsigned s0 = 1; e == cudaSuccess && s0 <= 0x7BFFu; s0 += 1024) {
+    const unsigned n_s = (0x7BFFu - s0 + 1 < 1024u) ? 0x7BFFu - s0 + 1 : 1024u;
+    const unsigned long long threads = static_cast<unsigned long long>(n_s) * 65536ull;
+    flexq::check_quantizer_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256>>>(
+        s0, n_s, d_count, d_first);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(mismatches, d_count, sizeof(unsigned long long), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(first_mismatch, d_first, 3 * sizeof(unsigned), cudaMemcpyDeviceToHost);
+  cudaFree(d_count);
+  if (e != cudaSuccess) return cuda_fail(e, "quantizer check");
+  return ok();
 }
 
 int flexq_debug_group_partials(int M, int N, int K, int group_size, const int8_t* Xq,

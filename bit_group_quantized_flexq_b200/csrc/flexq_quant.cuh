@@ -23,11 +23,43 @@ __device__ __forceinline__ __half group_scale(float amax, float qmax) {
   return __float2half_rn(__fdiv_rn(amax, qmax));
 }
 
-// One code, given the group's stored scale as FP32 (0 for a zero scale).
-__device__ __forceinline__ int quant_code(float x, float s, int qmax) {
+// One code by the defining route: IEEE FP32 division by the stored scale,
+// round half to even, clamp (0 for a zero scale).
+__device__ __forceinline__ int quant_code_div(float x, float s, int qmax) {
   if (s == 0.0f) return 0;
   int q = __float2int_rn(__fdiv_rn(x, s));
   return max(-qmax, min(qmax, q));
+}
+
+// The same code without a division, for FP16 x and FP16 s > 0 (passed as
+// FP32) and rs ~ 1/s.  Both are multiples of a power of two with at most 11
+// significant bits, so a quotient x/s that is not a half-integer lies at
+// least 2^-12 away from every half-integer, further than half an FP32 ulp at
+// the magnitudes a code can have (< 2^8): rounding the FP32 quotient to an
+// integer (half to even) therefore equals rounding the exact quotient.  The
+// estimate k0 = rint(x * rs) can only miss it at such a tie, by one.  The
+// residual r = x - k0 * s is exact (k0 * s has at most 19 significant bits
+// and lies within a factor 2 of x unless k0 = 0, where r = x), so comparing
+// |r| with s/2 decides exactly: beyond it, step towards r; at it (a tie),
+// step only if k0 is odd.
+__device__ __forceinline__ int quant_code_fast(float x, float s, float rs, int qmax) {
+  // estimates beyond +-(Q+2) only feed the clamp; bounding them keeps the
+  // integer arithmetic far from overflow
+  const float qb = static_cast<float>(qmax + 2);
+  const float k0 = fminf(fmaxf(rintf(x * rs), -qb), qb);
+  const float r = fmaf(-k0, s, x);
+  const float h = 0.5f * s;
+  const float ar = fabsf(r);
+  const int k = static_cast<int>(k0);
+  const bool step = ar > h || (ar == h && (k & 1));
+  const int q = step ? (r > 0.0f ? k + 1 : k - 1) : k;
+  return max(-qmax, min(qmax, q));
+}
+
+// One code, given the group's stored scale as FP32 (0 for a zero scale) and
+// its reciprocal estimate.
+__device__ __forceinline__ int quant_code(float x, float s, float rs, int qmax) {
+  return s == 0.0f ? 0 : quant_code_fast(x, s, rs, qmax);
 }
 
 // --------------------------------------------------------------------------
@@ -37,51 +69,64 @@ __device__ __forceinline__ int quant_code(float x, float s, int qmax) {
 template <int GS>
 __global__ void __launch_bounds__(256) quant_act_kernel(
     const uint4* __restrict__ X, uint2* __restrict__ Xq, __half* __restrict__ Xs,
-    long long chunks, int chunks_per_row, int ld_scales, int qmax) {
+    int M, int chunks_per_row, int rows_per_step, int ld_scales, int qmax) {
   constexpr int LANES = GS / 8;            // lanes per group
+  constexpr int U = 4;                     // independent 16-byte loads in flight per thread
   static_assert(LANES >= 4 && LANES <= 32, "group size 32..256");
   // X may be the output of the previous kernel of the stream, and Xq / Xs
   // may still be read by it: wait for it before touching either
   grid_launch_dependents();
   grid_wait_dependencies();
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  const long long first = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  // every lane of a warp runs the same number of iterations (the stride and
-  // the start are warp-aligned), so the shuffles below are always full-warp
-  const long long base_iters = (chunks + stride - 1) / stride;
+  // The grid covers rows_per_step whole rows per step (its thread count is a
+  // multiple of the row length in chunks), so each thread keeps one column c
+  // and advances by rows_per_step rows; a warp never straddles two rows in a
+  // way that splits a group, and every lane of a warp runs the same steps,
+  // so the shuffles below are always full-warp.
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  const int c = t % chunks_per_row;
+  const int row0 = t / chunks_per_row;
   const float fq = static_cast<float>(qmax);
-  for (long long it = 0; it < base_iters; ++it) {
-    const long long idx = first + it * stride;
-    const bool valid = idx < chunks;
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    if (valid) raw = __ldg(X + idx);
-    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
-    float v[8];
+  const int steps = (M + rows_per_step - 1) / rows_per_step;
+  for (int st0 = 0; st0 < steps; st0 += U) {
+    uint4 raw[U];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(h2[i]);
-      v[2 * i] = f.x;
-      v[2 * i + 1] = f.y;
+    for (int u = 0; u < U; ++u) {
+      const int row = row0 + (st0 + u) * rows_per_step;
+      raw[u] = make_uint4(0, 0, 0, 0);
+      if (st0 + u < steps && row < M)
+        raw[u] = __ldg(X + static_cast<long long>(row) * chunks_per_row + c);
     }
-    float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    for (int u = 0; u < U; ++u) {
+      if (st0 + u >= steps) break;           // uniform across the grid
+      const int row = row0 + (st0 + u) * rows_per_step;
+      const __half2* h2 = reinterpret_cast<const __half2*>(&raw[u]);
+      float v[8];
 #pragma unroll
-    for (int off = 1; off < LANES; off <<= 1)
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    const __half s16 = group_scale(amax, fq);
-    const float s = __half2float(s16);
-    uint32_t lo = 0, hi = 0;
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h2[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+      }
+      float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      lo |= (static_cast<uint32_t>(quant_code(v[i], s, qmax)) & 0xFFu) << (8 * i);
-      hi |= (static_cast<uint32_t>(quant_code(v[4 + i], s, qmax)) & 0xFFu) << (8 * i);
-    }
-    if (valid) {
-      Xq[idx] = make_uint2(lo, hi);
-      const long long row = idx / chunks_per_row;
-      const int c = static_cast<int>(idx - row * chunks_per_row);
-      if ((c % LANES) == 0) Xs[static_cast<long long>(c / LANES) * ld_scales + row] = s16;
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+      for (int off = 1; off < LANES; off <<= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      const __half s16 = group_scale(amax, fq);
+      const float sc = __half2float(s16);
+      const float rs = sc == 0.0f ? 0.0f : __frcp_rn(sc);
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        lo |= (static_cast<uint32_t>(quant_code(v[i], sc, rs, qmax)) & 0xFFu) << (8 * i);
+        hi |= (static_cast<uint32_t>(quant_code(v[4 + i], sc, rs, qmax)) & 0xFFu) << (8 * i);
+      }
+      if (row < M) {
+        Xq[static_cast<long long>(row) * chunks_per_row + c] = make_uint2(lo, hi);
+        if ((c % LANES) == 0) Xs[static_cast<long long>(c / LANES) * ld_scales + row] = s16;
+      }
     }
   }
 }
@@ -162,11 +207,12 @@ __global__ void __launch_bounds__(256) weight_pack_kernel(
       const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
       const int kk = k0 + 16 * blk + 8 * c;
       const float s = __half2float(Ws[static_cast<long long>(kk / gs) * N + n]);
+      const float rs = s == 0.0f ? 0.0f : __frcp_rn(s);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 f = __half22float2(h2[i]);
-        u[8 * c + 2 * i] = static_cast<uint32_t>(quant_code(f.x, s, 31)) & 0x3Fu;
-        u[8 * c + 2 * i + 1] = static_cast<uint32_t>(quant_code(f.y, s, 31)) & 0x3Fu;
+        u[8 * c + 2 * i] = static_cast<uint32_t>(quant_code(f.x, s, rs, 31)) & 0x3Fu;
+        u[8 * c + 2 * i + 1] = static_cast<uint32_t>(quant_code(f.y, s, rs, 31)) & 0x3Fu;
       }
     }
     pack_block(u, word[3 * blk], word[3 * blk + 1], word[3 * blk + 2]);
@@ -178,6 +224,36 @@ __global__ void __launch_bounds__(256) weight_pack_kernel(
     const int j = half_idx * 3 + jj;
     uint4* dst = reinterpret_cast<uint4*>(tile + (j * 128 + r) * 16);
     *dst = make_uint4(word[4 * jj], word[4 * jj + 1], word[4 * jj + 2], word[4 * jj + 3]);
+  }
+}
+
+// --------------------------------------------------------------------------
+// Test hook: for FP16 scale patterns [s_first, s_first + n_s) (positive,
+// finite) against every finite FP16 value x, counts the (x, s) pairs where
+// quant_code_fast differs from quant_code_div, for Q = 31 and Q = 127, and
+// records the first mismatch.  One thread per (x, s) pair.
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) check_quantizer_kernel(unsigned s_first, unsigned n_s,
+                                                              unsigned long long* mismatches,
+                                                              unsigned* first) {
+  const unsigned long long t = static_cast<unsigned long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= static_cast<unsigned long long>(n_s) * 65536ull) return;
+  const unsigned xb = static_cast<unsigned>(t & 0xFFFFu);
+  const unsigned sb = s_first + static_cast<unsigned>(t >> 16);
+  if ((xb & 0x7C00u) == 0x7C00u) return;                      // x infinite or NaN
+  const float x = __half2float(__ushort_as_half(static_cast<unsigned short>(xb)));
+  const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(sb)));
+  const float rs = __frcp_rn(s);
+  const int qs[2] = {31, 127};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    if (quant_code_fast(x, s, rs, qs[i]) != quant_code_div(x, s, qs[i])) {
+      if (atomicAdd(mismatches, 1ull) == 0ull) {
+        first[0] = xb;
+        first[1] = sb;
+        first[2] = static_cast<unsigned>(qs[i]);
+      }
+    }
   }
 }
 

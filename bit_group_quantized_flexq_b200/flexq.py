@@ -59,6 +59,8 @@ def lib():
             "flexq_gemm_static_scratch": (c_int, [c_int, c_int, c_int, c_int, c_int, c_void_p,
                                                   c_void_p, c_void_p, c_void_p, c_void_p,
                                                   c_void_p]),
+            "flexq_debug_check_quantizer": (c_int, [ctypes.POINTER(ctypes.c_ulonglong),
+                                                    ctypes.POINTER(ctypes.c_uint)]),
             "flexq_debug_group_partials": (c_int, [c_int, c_int, c_int, c_int, c_void_p,
                                                    c_void_p, c_void_p, c_void_p]),
             "flexq_gemm_plan": (c_int, [c_int, c_int, c_int, c_int,
@@ -233,6 +235,15 @@ def gemm_static_scratch(xq, xs, wp, ws, N, group_size, act_bits=6, out=None):
     _check(lib().flexq_gemm_static_scratch(M, N, K, group_size, act_bits, _ptr(xq), _ptr(xs),
                                            _ptr(wp), _ptr(ws), _ptr(out), _stream(xq)))
     return out
+
+
+def debug_check_quantizer():
+    """(mismatch count, (x bits, s bits, Q) of the first) of the GPU's fast
+    code rule against the IEEE-division rule over all FP16 (x, s > 0) pairs."""
+    n = ctypes.c_ulonglong(0)
+    first = (ctypes.c_uint * 3)()
+    _check(lib().flexq_debug_check_quantizer(ctypes.byref(n), first))
+    return n.value, tuple(first)
 
 
 def debug_group_partials(xq, wp, N, group_size, out=None):

@@ -193,6 +193,18 @@ int flexq_gemm_static_scratch(int M, int N, int K, int group_size, int act_bits,
                               void* Y_fp16, void* stream);
 
 /*
+ * flexq_debug_check_quantizer -- test hook: runs the GPU quantizer's
+ * division-free code rule against the IEEE-division rule (FP32 division by
+ * the stored FP16 scale, round half to even, clamp) on every pair of a
+ * finite FP16 value and a positive finite FP16 scale, for Q = 31 and
+ * Q = 127.  Writes the number of differing (x, s, Q) cases to *mismatches
+ * and the first one found ({x bits, s bits, Q}) to first_mismatch[0..2].
+ * Synchronous; allocates and frees its own small device buffer.
+ */
+int flexq_debug_check_quantizer(unsigned long long* mismatches,
+                                unsigned int* first_mismatch);
+
+/*
  * flexq_debug_group_partials -- exports the per-group int32 partials of the
  * GEMM above, computed by the same kernel mainloop (test hook).
  *   P  out, int32 [G, M, N]: P[g][m][n] = sum_{k in g} Xq[m,k] * Wq[n,k].

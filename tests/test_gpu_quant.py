@@ -95,3 +95,11 @@ def test_weight_quant_pack_llama_shape():
     qw, sw, dev = oracle_weight_device_form(w.numpy(), gs)
     assert np.array_equal(bits16(np16(flexq.weight_scales_view(ws))), bits16(sw))
     assert np.array_equal(np16(wp), dev)
+
+
+def test_fast_code_rule_equals_the_ieee_division_rule_exhaustively():
+    # every finite FP16 x against every positive finite FP16 scale, Q = 31 and
+    # Q = 127: the division-free rule the kernels use gives the same code as
+    # FP32 division + round half to even + clamp
+    n, first = flexq.debug_check_quantizer()
+    assert n == 0, f"{n} mismatches, first (x bits, s bits, Q) = {first}"
