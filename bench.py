@@ -422,29 +422,37 @@ def run_flexq(args, rank, world):
 
 def gemm_diagnostics(W, device, hbm_gbs, int8_peak_tops, reps=10):
     """Per-M GEMM-only times and roofline fractions (HBM bound for M <= 16,
-    tensor bound above).  Each GEMM runs `reps` times back to back; the
-    weights of the other layers stream in between, so reads stay cold."""
+    tensor bound above).  For each M, one CUDA graph holds `reps` rounds of
+    the seven GEMMs back to back (the other layers' weights stream in
+    between, so each GEMM reads its weights cold); events bracket the graph
+    replay, so host launch work is not timed."""
     import torch
     from bit_group_quantized_flexq_b200 import flexq
     out = []
+    stream = torch.cuda.Stream(device)
     for M in W.ms:
-        durs = {name: [] for (name, _, _, _, _) in W.w}
-        for _ in range(reps):
-            for (name, N, K, wp, ws) in W.w:
-                xq, xs = W.xq[(M, K)], W.xs[(M, K)]
-                e0 = torch.cuda.Event(enable_timing=True)
-                e1 = torch.cuda.Event(enable_timing=True)
-                e0.record()
-                flexq.gemm(xq, xs, wp, ws, N, GS, ACT_BITS, out=W.y[(M, name)])
-                e1.record()
-                durs[name].append((e0, e1))
+        def body():
+            for _ in range(reps):
+                for (name, N, K, wp, ws) in W.w:
+                    flexq.gemm(W.xq[(M, K)], W.xs[(M, K)], wp, ws, N, GS, ACT_BITS,
+                               out=W.y[(M, name)])
+        with torch.cuda.stream(stream):
+            body()                                # eager pass: sets attributes, workspace
+            torch.cuda.synchronize(device)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                body()
+            g.replay()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
         torch.cuda.synchronize(device)
-        t_us, bytes_, flops = 0.0, 0.0, 0.0
-        for (name, N, K, _, _) in W.w:
-            d = statistics.median(a.elapsed_time(b) for a, b in durs[name]) * 1e3
-            t_us += d
-            bytes_ += gemm_bytes(M, N, K)
-            flops += 2.0 * M * N * K
+        t_us = e0.elapsed_time(e1) * 1e3 / reps
+        del g
+        bytes_ = sum(gemm_bytes(M, N, K) for (_, N, K, _, _) in W.w)
+        flops = sum(2.0 * M * N * K for (_, N, K, _, _) in W.w)
         gbs = bytes_ / (t_us * 1e-6) / 1e9
         tops = flops / (t_us * 1e-6) / 1e12
         bound = "hbm" if M <= 16 else "tensor"
