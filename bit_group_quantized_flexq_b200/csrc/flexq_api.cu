@@ -7,6 +7,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -138,35 +139,68 @@ int max_split_for(int T) {
 // partial tiles of T x 128.  The counters never move, so calls of different
 // shapes can share one workspace without their partial tiles landing on
 // another shape's counters.
+int min_blocks_for(int T) {
+  switch (T) {
+    case 16: return flexq::GemmCfg<16>::kMinBlocks;
+    case 32: return flexq::GemmCfg<32>::kMinBlocks;
+    case 64: return flexq::GemmCfg<64>::kMinBlocks;
+    default: return flexq::GemmCfg<128>::kMinBlocks;
+  }
+}
+
 constexpr size_t kCounterBytes = 4096;
 constexpr long long kMaxSplitTiles = kCounterBytes / sizeof(unsigned);
 
 struct Plan {
   int T;
-  int split;
+  int split;             // K split of the split tiles (1: none)
+  long long n_full;      // output tiles run whole, first
+  long long n_split;     // output tiles split `split` ways, after them
   long long ctas;
 };
 
+// Tokens per tile follow M.  With fewer output tiles than CTA slots (SMs x
+// CTAs per SM) every tile is split along K to fill the machine; otherwise the
+// whole waves run unsplit and only the tiles of a partial last wave are split,
+// so that the last wave is as full as the others.
 Plan make_plan(int M, int N, int K, int gs, int sms, bool partials) {
   Plan p;
   const int units = K / 256;                          // K stages of the kernel
   p.T = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
-  const long long tiles = static_cast<long long>(N / 128) * ((M + p.T - 1) / p.T);
-  const long long slots = static_cast<long long>(sms) * (p.T <= 64 ? 2 : 1);
-  long long s = (slots + tiles / 2) / tiles;          // round(slots / tiles)
-  if (s < 1) s = 1;
-  if (s > max_split_for(p.T)) s = max_split_for(p.T);
-  if (s > units) s = units;
-  p.split = static_cast<int>(s);
   const int fT = g_force_tokens.load(), fS = g_force_split.load();
   if (fT == 16 || fT == 32 || fT == 64 || fT == 128) {
     if (fT >= p.T || fT >= M) p.T = fT;      // a tile must cover >= 1 token row
-    if (p.split > max_split_for(p.T)) p.split = max_split_for(p.T);
   }
-  if (fS >= 1 && fS <= max_split_for(p.T) && fS <= units) p.split = fS;
-  if (partials || tiles > kMaxSplitTiles) p.split = 1;
-  p.ctas = static_cast<long long>(p.split) * (N / 128) * ((M + p.T - 1) / p.T);
+  const long long tiles = static_cast<long long>(N / 128) * ((M + p.T - 1) / p.T);
+  const long long slots = static_cast<long long>(sms) * min_blocks_for(p.T);
+  const long long max_s = std::min<long long>(max_split_for(p.T), units);
+  long long s = 1, n_split = 0;
+  if (tiles < slots) {
+    s = (slots + tiles / 2) / tiles;                  // round(slots / tiles)
+    n_split = tiles;
+  } else if (tiles % slots) {
+    n_split = tiles % slots;                          // the partial last wave
+    s = (slots + n_split / 2) / n_split;
+  }
+  s = std::max<long long>(1, std::min(s, max_s));
+  if (fS >= 1 && fS <= max_split_for(p.T) && fS <= units) {
+    s = fS;                                           // forced: every tile split fS ways
+    n_split = tiles;
+  }
+  if (partials || s == 1 || n_split > kMaxSplitTiles) {
+    s = 1;
+    n_split = 0;
+  }
+  p.split = static_cast<int>(s);
+  p.n_split = n_split;
+  p.n_full = tiles - n_split;
+  p.ctas = p.n_full + p.n_split * p.split;
   return p;
+}
+
+size_t workspace_bytes_for(const Plan& p, int /*M*/, int /*N*/) {
+  if (p.split <= 1 || p.n_split == 0) return 0;
+  return kCounterBytes + static_cast<size_t>(p.n_split) * p.split * p.T * 128 * sizeof(float);
 }
 
 // ------------------------------------------------------------ tensor map --
@@ -230,15 +264,11 @@ int smem_bytes_for() {
   return 1024 + ctrl_offset_for<T>() + static_cast<int>(sizeof(flexq::GemmCtrl<T>));
 }
 
-size_t workspace_bytes_for(const Plan& p, int M, int N) {
-  if (p.split <= 1) return 0;
-  const size_t tiles = static_cast<size_t>(N / 128) * ((M + p.T - 1) / p.T);
-  return kCounterBytes + tiles * static_cast<size_t>(p.split) * p.T * 128 * sizeof(float);
-}
 
 template <int T, bool PARTIALS>
 int launch_gemm_t(DeviceState* st, const CUtensorMap& map, const CUtensorMap& map_sa,
-                  const CUtensorMap& map_sw, flexq::GemmArgs a, cudaStream_t stream) {
+                  const CUtensorMap& map_sw, flexq::GemmArgs a, long long grid_ctas,
+                  cudaStream_t stream) {
   using Cfg = flexq::GemmCfg<T>;
   auto kern = flexq::gemm_w6ax_kernel<T, PARTIALS>;
   const unsigned bit = 1u << ((T == 16 ? 0 : T == 32 ? 1 : T == 64 ? 2 : 3) + (PARTIALS ? 4 : 0));
@@ -253,8 +283,7 @@ int launch_gemm_t(DeviceState* st, const CUtensorMap& map, const CUtensorMap& ma
   }
   a.ctrl_offset = ctrl_offset_for<T>();
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(a.split), static_cast<unsigned>(a.N / 128),
-                     static_cast<unsigned>((a.M + T - 1) / T));
+  cfg.gridDim = dim3(static_cast<unsigned>(grid_ctas), 1, 1);
   cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes_for<T>());
   cfg.stream = stream;
@@ -292,13 +321,19 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
   const size_t need = workspace_bytes_for(plan, M, N);
   if (need > 0) {
     if (workspace == nullptr && workspace_bytes == 0) {
-      plan.split = 1;                      // no workspace: no K split
+      // no workspace: no K split (below)
     } else if (workspace == nullptr || workspace_bytes < need) {
       return fail(FLEXQ_ERR_INVALID_ARG, "workspace of %zu bytes at %p, the plan needs %zu",
                   workspace_bytes, workspace, need);
     } else if (!aligned16(workspace)) {
       return fail(FLEXQ_ERR_MISALIGNED, "workspace is not 16-byte aligned");
     }
+  }
+  if (plan.split > 1 && (workspace == nullptr || need == 0)) {   // run every tile whole
+    plan.split = 1;
+    plan.n_full += plan.n_split;
+    plan.n_split = 0;
+    plan.ctas = plan.n_full;
   }
   CUtensorMap map, map_sa, map_sw;
   if ((rc = encode_x_map(&map, Xq, M, K, plan.T))) return rc;
@@ -319,14 +354,17 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
   }
   a.status = st->status;
   a.wait_limit_ns = g_wait_limit_ns.load();
-  a.M = M; a.N = N; a.K = K; a.gs = gs; a.split = plan.split;
+  a.M = M; a.N = N; a.K = K; a.gs = gs;
+  a.tiles_n = N / 128;
+  a.n_full = static_cast<int>(plan.n_full);
+  a.split = plan.split;
   a.stall = g_inject_stall.exchange(0);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (plan.T) {
-    case 16: rc = partials ? launch_gemm_t<16, true>(st, map, map_sa, map_sw, a, s) : launch_gemm_t<16, false>(st, map, map_sa, map_sw, a, s); break;
-    case 32: rc = partials ? launch_gemm_t<32, true>(st, map, map_sa, map_sw, a, s) : launch_gemm_t<32, false>(st, map, map_sa, map_sw, a, s); break;
-    case 64: rc = partials ? launch_gemm_t<64, true>(st, map, map_sa, map_sw, a, s) : launch_gemm_t<64, false>(st, map, map_sa, map_sw, a, s); break;
-    default: rc = partials ? launch_gemm_t<128, true>(st, map, map_sa, map_sw, a, s) : launch_gemm_t<128, false>(st, map, map_sa, map_sw, a, s); break;
+    case 16: rc = partials ? launch_gemm_t<16, true>(st, map, map_sa, map_sw, a, plan.ctas, s) : launch_gemm_t<16, false>(st, map, map_sa, map_sw, a, plan.ctas, s); break;
+    case 32: rc = partials ? launch_gemm_t<32, true>(st, map, map_sa, map_sw, a, plan.ctas, s) : launch_gemm_t<32, false>(st, map, map_sa, map_sw, a, plan.ctas, s); break;
+    case 64: rc = partials ? launch_gemm_t<64, true>(st, map, map_sa, map_sw, a, plan.ctas, s) : launch_gemm_t<64, false>(st, map, map_sa, map_sw, a, plan.ctas, s); break;
+    default: rc = partials ? launch_gemm_t<128, true>(st, map, map_sa, map_sw, a, plan.ctas, s) : launch_gemm_t<128, false>(st, map, map_sa, map_sw, a, plan.ctas, s); break;
   }
   return rc ? rc : ok();
 }

@@ -60,7 +60,10 @@ struct GemmArgs {
   unsigned int* ws_cnt;    // split-K arrival counters [tiles], zero between calls
   unsigned int* status;    // device status word [4]
   unsigned long long wait_limit_ns;
-  int M, N, K, gs, split;
+  int M, N, K, gs;
+  int tiles_n;             // weight tiles along N (N / 128)
+  int n_full;              // output tiles 0 .. n_full-1 run whole (no K split) ...
+  int split;               // ... the later ones are split `split` ways along K
   int ctrl_offset;         // byte offset of the control block in smem
   int stall;               // test hook: withhold the first stage
 };
@@ -75,7 +78,7 @@ struct GemmCfg {
   static constexpr int kThreads = (6 + kEpiWarps) * 32;
   static constexpr int kStages = (T == 64) ? 2 : 3;
   static constexpr int kMinBlocks = (T <= 64) ? 2 : 1;
-  static constexpr int kMaxSplit = (T == 16) ? 8 : (T == 32) ? 6 : (T == 64) ? 4 : 2;
+  static constexpr int kMaxSplit = (T == 16) ? 8 : (T == 32) ? 6 : 4;
   static constexpr int kKStage = 2 * kKBlock;            // codes of K per stage
   static constexpr int kXsHalf = T * 128;                // one activation box
   static constexpr int kXsBytes = 2 * kXsHalf;
@@ -100,8 +103,6 @@ struct GemmCfg {
   static constexpr int kTmemCols = (kACol0 + kACols * kASlots <= 256) ? 256 : 512;
   static_assert(kACol0 + kACols * kASlots <= kTmemCols, "TMEM budget");
   static_assert(kMinBlocks == 1 || kTmemCols <= 256, "two CTAs per SM share 512 columns");
-  static constexpr int kLdChunk = (T == 64) ? 16 : kCols;   // TMEM columns per load batch
-  static_assert(kCols % kLdChunk == 0 && kLdChunk % 16 == 0, "epilogue column chunking");
 };
 
 template <int T>
@@ -219,16 +220,6 @@ __device__ __forceinline__ void unpack_block(uint32_t w0, uint32_t w1, uint32_t 
   out[3] = ((p2 * 4u + p1) * 4u + p0) * 4u;
 }
 
-template <int CH>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[CH]) {
-  static_assert(CH == 16 || CH == 32, "16 or 32 columns per load");
-  if constexpr (CH == 32) {
-    tmem_ld32(taddr, r);
-  } else {
-    tmem_ld16(taddr, r);
-  }
-}
-
 template <int T, bool PARTIALS>
 __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     gemm_w6ax_kernel(const __grid_constant__ CUtensorMap tmap_x,
@@ -253,10 +244,25 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   // for this grid before it reads anything this grid writes
   if (threadIdx.x == 0) grid_launch_dependents();
 
-  const int ks = blockIdx.x;            // K split index
-  const int nt = blockIdx.y;            // weight tile
-  const int mt = blockIdx.z;            // token tile
-  const int M = args.M, N = args.N, K = args.K, gs = args.gs, S = args.split;
+  // work unit -> output tile and K range: the first n_full units are whole
+  // tiles; after them every tile takes `split` consecutive units, one per K
+  // range (the plan splits only what would otherwise run as a partial last
+  // wave, or everything when there are fewer tiles than SMs)
+  const int unit = blockIdx.x;
+  int tile, ks, S;
+  if (unit < args.n_full) {
+    tile = unit;
+    ks = 0;
+    S = 1;
+  } else {
+    const int u = unit - args.n_full;
+    tile = args.n_full + u / args.split;
+    ks = u - (u / args.split) * args.split;
+    S = args.split;
+  }
+  const int nt = tile % args.tiles_n;   // weight tile (fastest: neighbours share the tokens)
+  const int mt = tile / args.tiles_n;   // token tile
+  const int M = args.M, N = args.N, K = args.K, gs = args.gs;
   const int KB = K / kKBlock;                         // 128-wide weight tiles
   const int units = K / Cfg::kKStage;                 // stages along K (gs | 256)
   const int u0 = static_cast<int>((static_cast<long long>(ks) * units) / S);
@@ -505,7 +511,6 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     if (q == 0 && lane == 0) FLEXQ_ROLE_DONE(2, nst);
   } else {
     // ------------------------------------------------------ epilogue -----
-    constexpr int CH = Cfg::kLdChunk;
     const int e = warp - 6;
     const int q = warp & 3;
     const int c = e >> 2;
@@ -546,42 +551,45 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         break;
       }
       tc_fence_after();
-      // drain the partials in chunks; the buffer is released right after the
-      // last chunk has been read, before that chunk's arithmetic
+      // two 16-column loads: the second is issued before the first chunk's
+      // arithmetic, so its latency hides behind it; the buffer is released
+      // once both have landed
+      static_assert(Cfg::kCols == 32 || Cfg::kCols == 16, "chunking");
+      constexpr int NC = Cfg::kCols / 16;
+      const uint32_t pcol = tmem + lane_base + Cfg::kPCol0 + pb.idx * T + col0;
+      uint32_t pv[NC][16];
+      tmem_ld16(pcol, pv[0]);
+      tmem_wait_ld();
+      if (NC == 2) tmem_ld16(pcol + 16, pv[NC - 1]);
 #pragma unroll
-      for (int ch = 0; ch < Cfg::kCols / CH; ++ch) {
-        uint32_t pv[CH];
-        tmem_ld_cols<CH>(tmem + lane_base + Cfg::kPCol0 + pb.idx * T + col0 + ch * CH, pv);
-        tmem_wait_ld();
-        if (ch == Cfg::kCols / CH - 1) {
+      for (int ch = 0; ch < NC; ++ch) {
+        if (ch == NC - 1) {
+          if (NC == 2) tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctrl->p_empty[pb.idx]);
         }
         if (PARTIALS) {
 #pragma unroll
-          for (int j = 0; j < CH; ++j) {
-            const int m = m_base + ch * CH + j;
+          for (int j = 0; j < 16; ++j) {
+            const int m = m_base + ch * 16 + j;
             if (m < M)
-              args.p[(static_cast<size_t>(g) * M + m) * N + n] =
-                  static_cast<int32_t>(pv[j]) >> 2;
+              args.p[(static_cast<size_t>(g) * M + m) * N + n] = static_cast<int32_t>(pv[ch][j]) >> 2;
           }
         } else {
-          // acc += float(P) * (sw/4 * sa), two columns per instruction; the
-          // FP16 x FP16 scale product is exact in FP32, the FMA rounds once
           const float2 swn2 = make_float2(swn, swn);
-          const float4* sa4 = reinterpret_cast<const float4*>(sa_w + ch * CH);
+          const float4* sa4 = reinterpret_cast<const float4*>(sa_w + ch * 16);
 #pragma unroll
-          for (int j = 0; j < CH; j += 4) {
+          for (int j = 0; j < 16; j += 4) {
             const float4 s4 = sa4[j / 4];
             const float2 s_lo = __fmul2_rn(swn2, make_float2(s4.x, s4.y));
             const float2 s_hi = __fmul2_rn(swn2, make_float2(s4.z, s4.w));
-            const float2 p_lo = make_float2(__int2float_rn(static_cast<int32_t>(pv[j])),
-                                            __int2float_rn(static_cast<int32_t>(pv[j + 1])));
-            const float2 p_hi = make_float2(__int2float_rn(static_cast<int32_t>(pv[j + 2])),
-                                            __int2float_rn(static_cast<int32_t>(pv[j + 3])));
-            acc[(ch * CH + j) / 2] = __ffma2_rn(p_lo, s_lo, acc[(ch * CH + j) / 2]);
-            acc[(ch * CH + j) / 2 + 1] = __ffma2_rn(p_hi, s_hi, acc[(ch * CH + j) / 2 + 1]);
+            const float2 p_lo = make_float2(__int2float_rn(static_cast<int32_t>(pv[ch][j])),
+                                            __int2float_rn(static_cast<int32_t>(pv[ch][j + 1])));
+            const float2 p_hi = make_float2(__int2float_rn(static_cast<int32_t>(pv[ch][j + 2])),
+                                            __int2float_rn(static_cast<int32_t>(pv[ch][j + 3])));
+            acc[(ch * 16 + j) / 2] = __ffma2_rn(p_lo, s_lo, acc[(ch * 16 + j) / 2]);
+            acc[(ch * 16 + j) / 2 + 1] = __ffma2_rn(p_hi, s_hi, acc[(ch * 16 + j) / 2 + 1]);
           }
         }
       }
@@ -617,8 +625,8 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     // last CTA of the output tile to arrive adds the `split` partials in
     // split order (the same order whichever CTA arrives last, so the result
     // is deterministic), writes the FP16 output and resets the counter.
-    const size_t tile = static_cast<size_t>(mt) * gridDim.y + nt;
-    float* part = args.ws_part + tile * static_cast<size_t>(S) * T * kTileRows;
+    const size_t st_idx = static_cast<size_t>(tile - args.n_full);     // split tile index
+    float* part = args.ws_part + st_idx * static_cast<size_t>(S) * T * kTileRows;
     if (is_epi) {
 #pragma unroll
       for (int j = 0; j < Cfg::kCols; ++j)
@@ -629,9 +637,9 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     __syncthreads();
     FLEXQ_CTA_TIME(6);
     if (threadIdx.x == 0) {
-      const unsigned old = atomicAdd(&args.ws_cnt[tile], 1u);
+      const unsigned old = atomicAdd(&args.ws_cnt[st_idx], 1u);
       const bool last = old == static_cast<unsigned>(S - 1);
-      if (last) args.ws_cnt[tile] = 0u;
+      if (last) args.ws_cnt[st_idx] = 0u;
       ctrl->is_last = last ? 1u : 0u;
     }
     __syncthreads();

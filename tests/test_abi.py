@@ -93,7 +93,15 @@ def test_plan_is_host_only_and_sane(L):
         t, s, c = flexq.plan(M, 4096, 4096, 128)
         assert t == T
         assert 1 <= s <= 8
-        assert c == s * (4096 // 128) * ((M + t - 1) // t)
+        tiles = (4096 // 128) * ((M + t - 1) // t)
+        if tiles < 148:                   # fewer tiles than SMs: every tile split
+            assert c == s * tiles
+        else:                             # whole waves unsplit, the last wave split
+            assert tiles <= c <= s * tiles
+    # M = 2048, N = K = 4096: 512 tiles = 3 waves of 148 + 68; those 68 split in 2
+    assert flexq.plan(2048, 4096, 4096, 128) == (128, 2, 444 + 2 * 68)
+    # N = 11008: 1376 tiles = 9 waves + 44; those 44 split in 3
+    assert flexq.plan(2048, 11008, 4096, 128) == (128, 3, 1332 + 3 * 44)
     t, s, c = flexq.plan(1, 4096, 4096, 128)
     assert s > 1                      # 32 weight tiles alone would idle most SMs
     t, s, c = flexq.plan(1, 4096, 256, 256)
@@ -104,10 +112,11 @@ def test_plan_is_host_only_and_sane(L):
 def test_workspace_size_follows_the_plan(L):
     # no K split: no workspace; a K split: FP32 partial tiles + one counter per tile
     assert flexq.gemm_workspace_bytes(2048, 4096, 4096, 128) == 0 or flexq.plan(2048, 4096, 4096, 128)[1] > 1
-    for M, N, K in [(1, 4096, 4096), (16, 11008, 4096), (5, 384, 4096)]:
+    for M, N, K in [(1, 4096, 4096), (16, 11008, 4096), (5, 384, 4096), (2048, 4096, 4096)]:
         t, s, c = flexq.plan(M, N, K, 128)
         tiles = (N // 128) * ((M + t - 1) // t)
-        want = 0 if s == 1 else 4096 + tiles * s * t * 128 * 4
+        n_split = (c - tiles) // (s - 1) if s > 1 else 0
+        want = 0 if s == 1 else 4096 + n_split * s * t * 128 * 4
         assert flexq.gemm_workspace_bytes(M, N, K, 128) == want
     assert flexq.gemm_workspace_bytes(0, 4096, 4096, 128) == 0
     assert flexq.gemm_workspace_bytes(4, 200, 4096, 128) == 0

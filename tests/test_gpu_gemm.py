@@ -219,3 +219,20 @@ def test_too_small_workspace_is_rejected():
     with pytest.raises(flexq.FlexQError) as ei:
         flexq.gemm(xq, xs, wp, ws, N, gs, 6, workspace_buf=small)
     assert ei.value.status == flexq.FLEXQ_ERR_INVALID_ARG
+
+
+def test_whole_waves_and_split_last_wave():
+    # 2 token tiles x 80 weight tiles = 160 output tiles: one whole wave on 148
+    # SMs runs unsplit and the 12 tiles of the last wave are split along K
+    M, N, K, gs, bits = 200, 10240, 1024, 128, 6
+    t, s, c = flexq.plan(M, N, K, gs)
+    assert (t, s) == (128, 4) and c == 148 + 4 * 12
+    seed = inputs.layer_seed("tail", M, N, K)
+    x = inputs.activations(M, K, seed=seed)
+    w = inputs.weights(N, K, seed=seed + 1)
+    wp, ws = flexq.quantize_weight(w.cuda(), gs)
+    y = np16(flexq.linear(x.cuda(), wp, ws, N, gs, bits))
+    rows = [0, 1, 127, 128, 150, 199]
+    qw, sw = orc.quantize_weight(w.numpy(), gs)
+    qa, sa = orc.quantize_act(x.numpy()[rows], gs, bits)
+    assert_within(y[rows], orc.gemm_fp64(qa, sa, qw, sw, gs), TOL)
