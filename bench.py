@@ -410,6 +410,8 @@ def run_flexq(args, rank, world):
                                       f"M={dominant_m}; events between graph launches")
     if diag:
         result["gemm_by_m"] = diag
+    if args.diag and rank == 0:
+        result["int8_library_context"] = int8_library_context(W, device, dominant_m)
     if args.e2e:
         result["e2e"] = run_e2e(W, args, device, world)
     if rank == 0 and world == 1 and args.cpu_baseline:
@@ -461,6 +463,41 @@ def gemm_diagnostics(W, device, hbm_gbs, int8_peak_tops, reps=10):
                     "TOPS": round(tops, 2), "bound": bound, "frac": round(frac, 4),
                     "plan": [list(flexq.plan(M, N, K, GS)) for (_, N, K, _, _) in W.w]})
     return out
+
+
+def int8_library_context(W, device, M, reps=20):
+    """Context only, never the target: the library int8 GEMM (torch._int_mm,
+    plain W8A8 without group scales) on this GPU at the dominant M's shapes,
+    and its rate on an 8192^3 problem (an on-box int8 tensor figure to set
+    beside the nominal ratio used for the roofline)."""
+    import torch
+
+    def time_mm(m, n, k):
+        a = torch.randint(-127, 128, (m, k), dtype=torch.int8, device=device)
+        b = torch.randint(-127, 128, (n, k), dtype=torch.int8, device=device).t()
+        for _ in range(3):
+            torch._int_mm(a, b)
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            torch._int_mm(a, b)
+        e1.record()
+        torch.cuda.synchronize(device)
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        return round(us, 2), round(2.0 * m * n * k / (us * 1e-6) / 1e12, 1)
+
+    try:
+        shapes = []
+        for (name, N, K, _, _) in W.w:
+            us, tops = time_mm(M, N, K)
+            shapes.append({"layer": name, "M": M, "N": N, "K": K, "us": us, "TOPS": tops})
+        us, tops = time_mm(8192, 8192, 8192)
+        return {"kernel": "torch._int_mm (int8 x int8 -> int32, no group scales)",
+                "layers": shapes, "int8_8192_cube_TOPS": tops}
+    except (RuntimeError, AttributeError) as exc:       # not available in this torch build
+        return {"unavailable": str(exc).splitlines()[0][:200]}
 
 
 def run_e2e(W, args, device, world):
