@@ -115,16 +115,36 @@ def aggregate(units_per_rank, world, t_max_s):
 
 # ----------------------------------------------------------------- clocks --
 class ClockSampler:
+    """SM clocks and throttle reasons of one GPU, polled every few
+    milliseconds from a thread through NVML while the timed region runs
+    (nvidia-smi's ~100 ms period can miss a region of a few tens of ms);
+    falls back to nvidia-smi when NVML is not importable."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.002
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.nvml = None
         self.lines = []
+        self.samples = []            # (sm_mhz, max_mhz, reasons bitmask)
+        self._stop = threading.Event()
+        self.thread = None
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.nvml = (pynvml, h)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:            # no NVML: sample with nvidia-smi instead
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
@@ -135,11 +155,26 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self.proc = None
 
+    def _poll(self):
+        pynvml, h = self.nvml
+        while not self._stop.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, self.max_mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.PERIOD_S)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
     def stop(self):
+        self._stop.set()
+        if self.nvml is not None:
+            self.thread.join(timeout=5)
+            return self.summary_nvml()
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -149,6 +184,19 @@ class ClockSampler:
             self.proc.kill()
         self.thread.join(timeout=5)
         return self.summary()
+
+    def summary_nvml(self):
+        pynvml, _ = self.nvml
+        if not self.samples:
+            return None
+        bits = {"hw_slowdown": getattr(pynvml, "nvmlClocksEventReasonHwSlowdown", 0x8),
+                "hw_thermal_slowdown": getattr(pynvml, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+                "sw_thermal_slowdown": getattr(pynvml, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+                "sw_power_cap": getattr(pynvml, "nvmlClocksEventReasonSwPowerCap", 0x4)}
+        reasons = sorted(n for n, b in bits.items() if any(r & b for _, _, r in self.samples))
+        return {"sm_mhz": statistics.median(sm for sm, _, _ in self.samples),
+                "sm_max_mhz": max(mx for _, mx, _ in self.samples),
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
 
     def summary(self):
         sm, smax, reasons = [], [], set()
@@ -168,7 +216,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi"}
 
 
 def measured_peaks():
@@ -322,7 +370,7 @@ def run_flexq(args, rank, world):
         torch.cuda.synchronize(device)
         clocks = ClockSampler(device.index if device.index is not None else 0)
         clocks.start()
-        time.sleep(0.3)                           # sampler up before timing
+        time.sleep(0.05)                          # sampler running before timing
         t0, t1 = new_event(), new_event()
         t0.record(stream)
         for i in range(args.steps):

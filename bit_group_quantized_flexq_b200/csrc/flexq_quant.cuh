@@ -117,12 +117,31 @@ __global__ void __launch_bounds__(256) quant_act_kernel(
       const __half s16 = group_scale(amax, fq);
       const float sc = __half2float(s16);
       const float rs = sc == 0.0f ? 0.0f : __frcp_rn(sc);
-      uint32_t lo = 0, hi = 0;
+      // Common path: rint(x * rs) is the code unless x/s is exactly a
+      // half-integer (see quant_code_fast), and a normal FP16 scale
+      // (>= 2^-14, rounded from absmax/Q with relative error <= 2^-11) keeps
+      // every |x/s| below Q + 1/2, so no clamp is needed.  A tie shows as an
+      // exact residual of s/2.  Warps that meet a tie or a subnormal or zero
+      // scale take the full rule for all their values.
+      const float h = 0.5f * sc;
+      float kf[8];
+      bool exact_path = !(sc >= 6.103515625e-05f);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        lo |= (static_cast<uint32_t>(quant_code(v[i], sc, rs, qmax)) & 0xFFu) << (8 * i);
-        hi |= (static_cast<uint32_t>(quant_code(v[4 + i], sc, rs, qmax)) & 0xFFu) << (8 * i);
+      for (int i = 0; i < 8; ++i) {
+        kf[i] = rintf(v[i] * rs);
+        exact_path |= fabsf(fmaf(-kf[i], sc, v[i])) == h;
       }
+      int q[8];
+      if (__any_sync(0xffffffffu, exact_path)) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = quant_code(v[i], sc, rs, qmax);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = __float2int_rn(kf[i]);
+      }
+      // low bytes of the codes, in order, two permutes per four codes
+      const uint32_t lo = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+      const uint32_t hi = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
       if (row < M) {
         Xq[static_cast<long long>(row) * chunks_per_row + c] = make_uint2(lo, hi);
         if ((c % LANES) == 0) Xs[static_cast<long long>(c / LANES) * ld_scales + row] = s16;
