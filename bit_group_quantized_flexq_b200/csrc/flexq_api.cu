@@ -175,12 +175,14 @@ Plan make_plan(int M, int N, int K, int gs, int sms, bool partials) {
   const long long slots = static_cast<long long>(sms) * min_blocks_for(p.T);
   const long long max_s = std::min<long long>(max_split_for(p.T), units);
   long long s = 1, n_split = 0;
+  // the split never makes the split tiles' units exceed one wave of slots:
+  // a second, partial wave costs more than the split saves
   if (tiles < slots) {
-    s = (slots + tiles / 2) / tiles;                  // round(slots / tiles)
+    s = slots / tiles;
     n_split = tiles;
   } else if (tiles % slots) {
     n_split = tiles % slots;                          // the partial last wave
-    s = (slots + n_split / 2) / n_split;
+    s = slots / n_split;
   }
   s = std::max<long long>(1, std::min(s, max_s));
   if (fS >= 1 && fS <= max_split_for(p.T) && fS <= units) {

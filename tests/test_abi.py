@@ -106,6 +106,11 @@ def test_plan_is_host_only_and_sane(L):
     assert s > 1                      # 32 weight tiles alone would idle most SMs
     t, s, c = flexq.plan(1, 4096, 256, 256)
     assert s == 1                     # one group: nothing to split
+    # the split units never exceed one wave of CTA slots (2 per SM at T = 16)
+    for N, K in [(8192, 8192), (11008, 4096), (4096, 11008), (28672, 8192)]:
+        t, s, c = flexq.plan(1, N, K, 128)
+        assert c <= 2 * 148
+    assert flexq.plan(1, 8192, 8192, 128) == (16, 4, 256)
     assert flexq.plan(0, 256, 256, 128) == (0, 0, 0)
 
 
