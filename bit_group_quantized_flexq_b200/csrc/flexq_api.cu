@@ -168,9 +168,7 @@ Plan make_plan(int M, int N, int K, int gs, int sms, bool partials) {
   const int units = K / 256;                          // K stages of the kernel
   p.T = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
   const int fT = g_force_tokens.load(), fS = g_force_split.load();
-  if (fT == 16 || fT == 32 || fT == 64 || fT == 128) {
-    if (fT >= p.T || fT >= M) p.T = fT;      // a tile must cover >= 1 token row
-  }
+  if (fT == 16 || fT == 32 || fT == 64 || fT == 128) p.T = fT;   // any width: more or fewer token tiles
   const long long tiles = static_cast<long long>(N / 128) * ((M + p.T - 1) / p.T);
   const long long slots = static_cast<long long>(sms) * min_blocks_for(p.T);
   const long long max_s = std::min<long long>(max_split_for(p.T), units);
