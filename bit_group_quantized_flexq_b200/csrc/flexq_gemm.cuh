@@ -520,34 +520,40 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const int m_base = mt * T + col0;
     FLEXQ_ROLE_CLOCK;
+    // groups in octets (the scale ring's unit): the eight groups of an octet
+    // are unrolled, so their scale offsets are compile-time constants and the
+    // ring slot and its release happen once per octet
     RingPos<NB> pb;
-    for (int lg = 0; lg < ngroups; ++lg) {
-      const int g = g0 + lg;
-      const int gi = lg & 7;
-      const int sc_slot = (lg >> 3) % Cfg::kScSlots;
-      const uint8_t* sc = sc_ring + sc_slot * Cfg::kScSlotBytes;
-      float swn = 0.0f;
+    RingPos<Cfg::kScSlots> sp;                       // scale-ring slot of the octet
+    bool failed = false;
+    for (int lo = 0; lo < ngroups && !failed; lo += 8) {
+      const uint8_t* sc = sc_ring + sp.idx * Cfg::kScSlotBytes;
+      const __half* sw_h = reinterpret_cast<const __half*>(sc + Cfg::kScSaBytes);
       if (!PARTIALS) {
-        if (gi == 0) {
-          if (!FLEXQ_WAIT(warp_wait(&ctrl->s_full[sc_slot], ((lg >> 3) / Cfg::kScSlots) & 1, lim))) {
-            if (lane == 0) record_status(args.status, kStatusTimeout, 5);
-            break;
-          }
-          // this warp's tokens of the octet, FP16 -> FP32, into its own buffer
-          const __half* sa_h = reinterpret_cast<const __half*>(sc);
-#pragma unroll
-          for (int idx = lane; idx < 8 * Cfg::kCols; idx += 32) {
-            const int gg = idx / Cfg::kCols, j = idx - gg * Cfg::kCols;
-            ctrl->sa[e][gg][j] = __half2float(sa_h[gg * T + col0 + j]);
-          }
-          __syncwarp();
+        if (!FLEXQ_WAIT(warp_wait(&ctrl->s_full[sp.idx], sp.phase, lim))) {
+          if (lane == 0) record_status(args.status, kStatusTimeout, 5);
+          break;
         }
-        const __half* sw_h = reinterpret_cast<const __half*>(sc + Cfg::kScSaBytes);
-        swn = __half2float(sw_h[gi * kTileRows + row]) * 0.25f;   // TMEM holds 4 * code
+        // this warp's tokens of the octet, FP16 -> FP32, into its own buffer
+        const __half* sa_h = reinterpret_cast<const __half*>(sc);
+#pragma unroll
+        for (int idx = lane; idx < 8 * Cfg::kCols; idx += 32) {
+          const int gg = idx / Cfg::kCols, j = idx - gg * Cfg::kCols;
+          ctrl->sa[e][gg][j] = __half2float(sa_h[gg * T + col0 + j]);
+        }
+        __syncwarp();
       }
+#pragma unroll
+      for (int gi = 0; gi < 8; ++gi) {
+      const int lg = lo + gi;
+      if (lg >= ngroups) break;
+      const int g = g0 + lg;
+      float swn = 0.0f;
+      if (!PARTIALS) swn = __half2float(sw_h[gi * kTileRows + row]) * 0.25f;
       const float* sa_w = ctrl->sa[e][gi];
       if (!FLEXQ_WAIT(warp_wait(&ctrl->p_full[pb.idx], pb.phase, lim))) {
         if (lane == 0) record_status(args.status, kStatusTimeout, 4);
+        failed = true;
         break;
       }
       tc_fence_after();
@@ -593,11 +599,13 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
           }
         }
       }
-      if (!PARTIALS && (gi == 7 || lg == ngroups - 1)) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctrl->s_empty[sc_slot]);
-      }
       pb.next();
+      }
+      if (!PARTIALS && !failed) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->s_empty[sp.idx]);
+      }
+      sp.next();
     }
     if (e == 0 && lane == 0) FLEXQ_ROLE_DONE(3, ngroups);
   }
