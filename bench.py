@@ -460,6 +460,7 @@ def run_flexq(args, rank, world):
         result["gemm_by_m"] = diag
     if args.diag and rank == 0:
         result["int8_library_context"] = int8_library_context(W, device, dominant_m)
+        result["act_quant"] = act_quant_diagnostics(device, hbm)
     if args.e2e:
         result["e2e"] = run_e2e(W, args, device, world)
     if rank == 0 and world == 1 and args.cpu_baseline:
@@ -510,6 +511,43 @@ def gemm_diagnostics(W, device, hbm_gbs, int8_peak_tops, reps=10):
         out.append({"M": M, "gemm_us": round(t_us, 2), "GB/s": round(gbs, 1),
                     "TOPS": round(tops, 2), "bound": bound, "frac": round(frac, 4),
                     "plan": [list(flexq.plan(M, N, K, GS)) for (_, N, K, _, _) in W.w]})
+    return out
+
+
+def act_quant_diagnostics(device, hbm_gbs, K=8192, ms=(1, 2048, 16384), reps=20):
+    """The activation quantizer alone on FP16 [M, 8192] inputs with the
+    workload's outlier channels (the sweep configuration's separate timing):
+    device time per call from a CUDA graph of `reps` calls, and its HBM
+    roofline at 2 B read + 1 B written per element + 2 B per group scale."""
+    import torch
+    from bit_group_quantized_flexq_b200 import flexq, inputs
+    out = []
+    stream = torch.cuda.Stream(device)
+    for M in ms:
+        x = inputs.activations(M, K, outlier_frac=0.005, outlier_scale=50.0,
+                               seed=inputs.layer_seed("act-sweep", M, K)).to(device)
+        xq = torch.empty(M, K, dtype=torch.int8, device=device)
+        xs = torch.empty(K // GS, flexq.act_scales_ld(M), dtype=torch.float16, device=device)
+        with torch.cuda.stream(stream):
+            flexq.quantize_act(x, GS, ACT_BITS, out=(xq, xs))
+            torch.cuda.synchronize(device)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(reps):
+                    flexq.quantize_act(x, GS, ACT_BITS, out=(xq, xs))
+            g.replay()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        del g
+        nbytes = 3.0 * M * K + 2.0 * M * K / GS
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out.append({"M": M, "K": K, "us": round(us, 2), "GB/s": round(gbs, 1),
+                    "bound": "hbm", "frac": round(gbs / hbm_gbs, 4)})
     return out
 
 
