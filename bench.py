@@ -277,7 +277,17 @@ class Layers:
         torch.cuda.synchronize(device)
 
     def launches_per_step(self):
-        return 2 * len(self.ms) * len(self.w)
+        """Kernel launches of one step: the dominant M runs the quantizer and
+        the GEMM as separate launches (timed apart); the other M run each
+        layer through flexq.linear (one launch where it quantizes inside the
+        GEMM, two otherwise)."""
+        from bit_group_quantized_flexq_b200 import flexq
+        dominant = max(self.ms)
+        n = 0
+        for M in self.ms:
+            for (_, N, K, _, _) in self.w:
+                n += 2 if M == dominant else flexq.linear_launches(M, N, K, GS)
+        return n
 
     def quant(self, M, layer):
         from bit_group_quantized_flexq_b200 import flexq
@@ -290,10 +300,14 @@ class Layers:
         flexq.gemm(self.xq[(M, K)], self.xs[(M, K)], wp, ws, N, GS, ACT_BITS,
                    out=self.y[(M, name)])
 
+    def linear(self, M, layer):
+        from bit_group_quantized_flexq_b200 import flexq
+        name, N, K, wp, ws = layer
+        flexq.linear(self.x[(M, K)], wp, ws, N, GS, ACT_BITS, out=self.y[(M, name)])
+
     def run_m(self, M):
         for layer in self.w:
-            self.quant(M, layer)
-            self.gemm(M, layer)
+            self.linear(M, layer)
 
     def step(self):
         for M in self.ms:
@@ -471,46 +485,75 @@ def run_flexq(args, rank, world):
     runners.clear()
 
 
+def linear_bytes(M, N, K, gs=GS):
+    """Algorithmic HBM bytes of one whole linear layer from FP16 activations:
+    packed weights, weight scales, FP16 activations read once, FP16 output."""
+    return 0.75 * N * K + 2.0 * N * K / gs + 2.0 * M * K + 2.0 * M * N
+
+
+def _graph_time_us(body, device, stream, reps):
+    """Device time of one `body()` from a CUDA graph of `reps` bodies."""
+    import torch
+    with torch.cuda.stream(stream):
+        body()                                    # eager pass: sets attributes, workspace
+        torch.cuda.synchronize(device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(reps):
+                body()
+        g.replay()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(device)
+    t_us = e0.elapsed_time(e1) * 1e3 / reps
+    del g
+    return t_us
+
+
 def gemm_diagnostics(W, device, hbm_gbs, int8_peak_tops, reps=10):
-    """Per-M GEMM-only times and roofline fractions (HBM bound for M <= 16,
-    tensor bound above).  For each M, one CUDA graph holds `reps` rounds of
-    the seven GEMMs back to back (the other layers' weights stream in
-    between, so each GEMM reads its weights cold); events bracket the graph
-    replay, so host launch work is not timed."""
+    """Per-M times and roofline fractions (HBM bound for M <= 16, tensor bound
+    above) of the seven layers, each timed from a CUDA graph that holds `reps`
+    rounds of them back to back (the other layers' weights stream in between,
+    so each launch reads its weights cold); events bracket the graph replay,
+    so host launch work is not timed.  `gemm_*`: the GEMM alone on quantized
+    activations; `linear_*`: the whole layer from FP16 activations through
+    flexq.linear (one launch with quantization inside the GEMM for batches of
+    at most 2 tokens, the quantizer and the GEMM otherwise)."""
     import torch
     from bit_group_quantized_flexq_b200 import flexq
     out = []
     stream = torch.cuda.Stream(device)
     for M in W.ms:
-        def body():
-            for _ in range(reps):
-                for (name, N, K, wp, ws) in W.w:
-                    flexq.gemm(W.xq[(M, K)], W.xs[(M, K)], wp, ws, N, GS, ACT_BITS,
-                               out=W.y[(M, name)])
-        with torch.cuda.stream(stream):
-            body()                                # eager pass: sets attributes, workspace
-            torch.cuda.synchronize(device)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                body()
-            g.replay()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            g.replay()
-            e1.record(stream)
-        torch.cuda.synchronize(device)
-        t_us = e0.elapsed_time(e1) * 1e3 / reps
-        del g
-        bytes_ = sum(gemm_bytes(M, N, K) for (_, N, K, _, _) in W.w)
+        for layer in W.w:
+            W.quant(M, layer)                     # the GEMM's quantized inputs
+
+        def gemm_body():
+            for (name, N, K, wp, ws) in W.w:
+                flexq.gemm(W.xq[(M, K)], W.xs[(M, K)], wp, ws, N, GS, ACT_BITS,
+                           out=W.y[(M, name)])
+
+        def linear_body():
+            for layer in W.w:
+                W.linear(M, layer)
+
+        t_us = _graph_time_us(gemm_body, device, stream, reps)
+        l_us = _graph_time_us(linear_body, device, stream, reps)
         flops = sum(2.0 * M * N * K for (_, N, K, _, _) in W.w)
-        gbs = bytes_ / (t_us * 1e-6) / 1e9
-        tops = flops / (t_us * 1e-6) / 1e12
         bound = "hbm" if M <= 16 else "tensor"
-        frac = gbs / hbm_gbs if bound == "hbm" else tops / int8_peak_tops
-        out.append({"M": M, "gemm_us": round(t_us, 2), "GB/s": round(gbs, 1),
-                    "TOPS": round(tops, 2), "bound": bound, "frac": round(frac, 4),
-                    "plan": [list(flexq.plan(M, N, K, GS)) for (_, N, K, _, _) in W.w]})
+        row = {"M": M, "bound": bound}
+        for key, us, nbytes in (("gemm", t_us, sum(gemm_bytes(M, N, K) for (_, N, K, _, _) in W.w)),
+                                ("linear", l_us, sum(linear_bytes(M, N, K) for (_, N, K, _, _) in W.w))):
+            gbs = nbytes / (us * 1e-6) / 1e9
+            tops = flops / (us * 1e-6) / 1e12
+            row[f"{key}_us"] = round(us, 2)
+            row[f"{key}_GB/s"] = round(gbs, 1)
+            row[f"{key}_TOPS"] = round(tops, 2)
+            row[f"{key}_frac"] = round(gbs / hbm_gbs if bound == "hbm" else tops / int8_peak_tops, 4)
+        row["plan"] = [list(flexq.plan(M, N, K, GS)) for (_, N, K, _, _) in W.w]
+        out.append(row)
     return out
 
 
@@ -602,8 +645,7 @@ def run_e2e(W, args, device, world):
         for M in W.ms:
             for (name, N, K, wp, ws) in W.w:
                 dx[(M, K)].copy_(hx[(M, K)], non_blocking=True)
-                flexq.linear(dx[(M, K)], wp, ws, N, GS, ACT_BITS,
-                             xq_out=(W.xq[(M, K)], W.xs[(M, K)]), y_out=W.y[(M, name)])
+                flexq.linear(dx[(M, K)], wp, ws, N, GS, ACT_BITS, out=W.y[(M, name)])
                 hy[(M, name)].copy_(W.y[(M, name)], non_blocking=True)
 
     for _ in range(args.warmup):

@@ -55,6 +55,7 @@ std::atomic<int> g_force_tokens{0};
 std::atomic<int> g_force_split{0};
 std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
 std::atomic<int> g_inject_stall{0};
+std::atomic<int> g_force_linear_route{0};   // 0 by plan, 1 fused quantization, 2 separate quantizer
 
 // ---------------------------------------------------------- device state --
 constexpr int kMaxDevices = 64;
@@ -259,33 +260,42 @@ int ctrl_offset_for() {
   return (flexq::GemmCfg<T>::kMainBytes + 15) & ~15;
 }
 
+// the fused activation quantizer's block (barriers and scale slots) follows
+// the control block
 template <int T>
+int fq_offset_for() {
+  return (ctrl_offset_for<T>() + static_cast<int>(sizeof(flexq::GemmCtrl<T>)) + 15) & ~15;
+}
+
+template <int T, bool FUSEDQ = false>
 int smem_bytes_for() {
+  if (FUSEDQ) return 1024 + fq_offset_for<T>() + flexq::FusedQLayout<T>::kBytes;
   return 1024 + ctrl_offset_for<T>() + static_cast<int>(sizeof(flexq::GemmCtrl<T>));
 }
 
-
-template <int T, bool PARTIALS>
+template <int T, bool PARTIALS, bool FUSEDQ = false>
 int launch_gemm_t(DeviceState* st, const CUtensorMap& map, const CUtensorMap& map_sa,
                   const CUtensorMap& map_sw, flexq::GemmArgs a, long long grid_ctas,
                   cudaStream_t stream) {
   using Cfg = flexq::GemmCfg<T>;
-  auto kern = flexq::gemm_w6ax_kernel<T, PARTIALS>;
-  const unsigned bit = 1u << ((T == 16 ? 0 : T == 32 ? 1 : T == 64 ? 2 : 3) + (PARTIALS ? 4 : 0));
+  auto kern = flexq::gemm_w6ax_kernel<T, PARTIALS, FUSEDQ>;
+  const unsigned bit = 1u << ((T == 16 ? 0 : T == 32 ? 1 : T == 64 ? 2 : 3) + (PARTIALS ? 4 : 0) +
+                              (FUSEDQ ? 8 : 0));
+  const int smem = smem_bytes_for<T, FUSEDQ>();
   {
     std::lock_guard<std::mutex> lock(g_dev_mutex);
     if (!(st->attr_mask & bit)) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           smem_bytes_for<T>());
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
       st->attr_mask |= bit;
     }
   }
   a.ctrl_offset = ctrl_offset_for<T>();
+  a.fq_offset = FUSEDQ ? fq_offset_for<T>() : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid_ctas), 1, 1);
   cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes_for<T>());
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
   // programmatic stream serialization: the kernel may start while the
   // previous kernel of the stream finishes (it prefetches its weights, then
@@ -297,6 +307,29 @@ int launch_gemm_t(DeviceState* st, const CUtensorMap& map, const CUtensorMap& ma
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map, map_sa, map_sw, a);
   if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
+  return FLEXQ_OK;
+}
+
+// The caller's split-K workspace against the plan: none (NULL, 0 bytes)
+// runs every tile whole; one too small for the plan is an error.
+int apply_workspace(Plan* plan, int M, int N, void* workspace, size_t workspace_bytes) {
+  const size_t need = workspace_bytes_for(*plan, M, N);
+  if (need > 0) {
+    if (workspace == nullptr && workspace_bytes == 0) {
+      // no workspace: no K split (below)
+    } else if (workspace == nullptr || workspace_bytes < need) {
+      return fail(FLEXQ_ERR_INVALID_ARG, "workspace of %zu bytes at %p, the plan needs %zu",
+                  workspace_bytes, workspace, need);
+    } else if (!aligned16(workspace)) {
+      return fail(FLEXQ_ERR_MISALIGNED, "workspace is not 16-byte aligned");
+    }
+  }
+  if (plan->split > 1 && (workspace == nullptr || need == 0)) {   // run every tile whole
+    plan->split = 1;
+    plan->n_full += plan->n_split;
+    plan->n_split = 0;
+    plan->ctas = plan->n_full;
+  }
   return FLEXQ_OK;
 }
 
@@ -318,23 +351,7 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
   Plan plan = make_plan(M, N, K, gs, st->sms, partials);
-  const size_t need = workspace_bytes_for(plan, M, N);
-  if (need > 0) {
-    if (workspace == nullptr && workspace_bytes == 0) {
-      // no workspace: no K split (below)
-    } else if (workspace == nullptr || workspace_bytes < need) {
-      return fail(FLEXQ_ERR_INVALID_ARG, "workspace of %zu bytes at %p, the plan needs %zu",
-                  workspace_bytes, workspace, need);
-    } else if (!aligned16(workspace)) {
-      return fail(FLEXQ_ERR_MISALIGNED, "workspace is not 16-byte aligned");
-    }
-  }
-  if (plan.split > 1 && (workspace == nullptr || need == 0)) {   // run every tile whole
-    plan.split = 1;
-    plan.n_full += plan.n_split;
-    plan.n_split = 0;
-    plan.ctas = plan.n_full;
-  }
+  if ((rc = apply_workspace(&plan, M, N, workspace, workspace_bytes))) return rc;
   CUtensorMap map, map_sa, map_sw;
   if ((rc = encode_x_map(&map, Xq, M, K, plan.T))) return rc;
   memset(&map_sa, 0, sizeof(map_sa));
@@ -366,6 +383,96 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
     case 64: rc = partials ? launch_gemm_t<64, true>(st, map, map_sa, map_sw, a, plan.ctas, s) : launch_gemm_t<64, false>(st, map, map_sa, map_sw, a, plan.ctas, s); break;
     default: rc = partials ? launch_gemm_t<128, true>(st, map, map_sa, map_sw, a, plan.ctas, s) : launch_gemm_t<128, false>(st, map, map_sa, map_sw, a, plan.ctas, s); break;
   }
+  return rc ? rc : ok();
+}
+
+// ------------------------------------------------------- linear layers --
+// A linear layer from FP16 activations: quantize them (bits 6 or 8), then the
+// group GEMM.  Batches of at most kFusedMaxM tokens (on 16-token tiles)
+// quantize inside the GEMM (one launch): there the in-kernel quantization,
+// whose rows each unpack warp takes one after another, costs no more than a
+// separate quantizer launch ahead of the GEMM; larger batches run the
+// activation quantizer first, its codes and scales in the caller's workspace
+// after the GEMM's region, whose arrival counters keep their fixed place at
+// the start.
+constexpr int kFusedMaxM = 2;
+
+bool linear_fused(const Plan& p, int M) {
+  const int route = g_force_linear_route.load();
+  if (p.T != 16) return false;
+  return route == 1 || (route == 0 && M <= kFusedMaxM);
+}
+
+struct LinearLayout {
+  bool fused;
+  size_t gemm_bytes;     // GEMM region from offset 0 (counters, partial tiles)
+  size_t xq_off, xs_off; // separate quantizer: codes [M, K] and scales [G][ld]
+  size_t total;
+};
+
+LinearLayout linear_layout(const Plan& p, int M, int N, int K, int gs) {
+  LinearLayout L = {};
+  L.fused = linear_fused(p, M);
+  L.gemm_bytes = workspace_bytes_for(p, M, N);
+  if (L.fused) {
+    L.total = L.gemm_bytes;
+    return L;
+  }
+  const size_t head = std::max(L.gemm_bytes, kCounterBytes);
+  L.xq_off = (head + 255) & ~static_cast<size_t>(255);
+  L.xs_off = (L.xq_off + static_cast<size_t>(M) * K + 255) & ~static_cast<size_t>(255);
+  L.total = L.xs_off + static_cast<size_t>(K / gs) * act_scales_ld(M) * sizeof(__half);
+  return L;
+}
+
+int linear_common(int M, int N, int K, int gs, int bits, const void* X, const void* Wp,
+                  const void* Ws, void* Y, void* workspace, size_t workspace_bytes, void* stream) {
+  if (bits != 6 && bits != 8) return fail(FLEXQ_ERR_INVALID_ARG, "bits=%d is not 6 or 8", bits);
+  int rc = check_gemm_shape(M, N, K, gs);
+  if (rc) return rc;
+  if (M == 0) return ok();               // empty batch: nothing to read or write
+  const void* ptrs[] = {X, Wp, Ws, Y};
+  const char* names[] = {"X_fp16", "Wq_packed", "W_scales", "Y"};
+  if ((rc = check_ptrs(4, ptrs, names))) return rc;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  Plan plan = make_plan(M, N, K, gs, st->sms, false);
+  const LinearLayout L = linear_layout(plan, M, N, K, gs);
+  if (!L.fused) {
+    if (workspace == nullptr || workspace_bytes < L.total)
+      return fail(FLEXQ_ERR_INVALID_ARG,
+                  "workspace of %zu bytes at %p: this shape quantizes its activations "
+                  "separately and needs %zu", workspace_bytes, workspace, L.total);
+    if (!aligned16(workspace)) return fail(FLEXQ_ERR_MISALIGNED, "workspace is not 16-byte aligned");
+    int8_t* xq = reinterpret_cast<int8_t*>(static_cast<char*>(workspace) + L.xq_off);
+    void* xs = static_cast<char*>(workspace) + L.xs_off;
+    if ((rc = flexq_quantize_act(M, K, gs, bits, X, xq, xs, stream))) return rc;
+    return gemm_common(M, N, K, gs, xq, xs, Wp, Ws, Y, nullptr, false, workspace, L.xq_off,
+                       stream);
+  }
+  if ((rc = apply_workspace(&plan, M, N, workspace, workspace_bytes))) return rc;
+  CUtensorMap map_x, map_sa, map_sw;     // activations and their scales: read by the kernel itself
+  memset(&map_x, 0, sizeof(map_x));
+  memset(&map_sa, 0, sizeof(map_sa));
+  if ((rc = encode_scale_map(&map_sw, Ws, N, N, K / gs, 128))) return rc;
+  flexq::GemmArgs a = {};
+  a.wp = static_cast<const uint8_t*>(Wp);
+  a.y = static_cast<__half*>(Y);
+  a.x = static_cast<const __half*>(X);
+  a.qmax = bits == 6 ? 31 : 127;
+  if (plan.split > 1) {
+    a.ws_cnt = static_cast<unsigned int*>(workspace);
+    a.ws_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kCounterBytes);
+  }
+  a.status = st->status;
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  a.M = M; a.N = N; a.K = K; a.gs = gs;
+  a.tiles_n = N / 128;
+  a.n_full = static_cast<int>(plan.n_full);
+  a.split = plan.split;
+  a.stall = g_inject_stall.exchange(0);
+  rc = launch_gemm_t<16, false, true>(st, map_x, map_sa, map_sw, a, plan.ctas,
+                                      static_cast<cudaStream_t>(stream));
   return rc ? rc : ok();
 }
 
@@ -560,6 +667,40 @@ int flexq_gemm_static_scratch(int M, int N, int K, int group_size, int act_bits,
   }
   return gemm_common(M, N, K, group_size, Xq, X_scales, Wq_packed, W_scales, Y_fp16, nullptr,
                      false, scratch, kStaticScratchBytes, stream);
+}
+
+size_t flexq_linear_workspace_bytes(int M, int N, int K, int group_size) {
+  if (M <= 0 || N <= 0 || K <= 0 || N % 128 || K % 256 || !valid_gs(group_size) || K % group_size)
+    return 0;
+  const Plan p = make_plan(M, N, K, group_size, sm_count_or_default(), false);
+  return linear_layout(p, M, N, K, group_size).total;
+}
+
+int flexq_linear_launches(int M, int N, int K, int group_size) {
+  if (M <= 0 || N <= 0 || K <= 0 || N % 128 || K % 256 || !valid_gs(group_size) || K % group_size)
+    return 0;
+  const Plan p = make_plan(M, N, K, group_size, sm_count_or_default(), false);
+  return linear_layout(p, M, N, K, group_size).fused ? 1 : 2;
+}
+
+int flexq_debug_force_linear_route(int route) {
+  if (route < 0 || route > 2) return fail(FLEXQ_ERR_INVALID_ARG, "route %d not in {0, 1, 2}", route);
+  g_force_linear_route.store(route);
+  return ok();
+}
+
+int flexq_linear_w6a6(int M, int N, int K, int group_size, const void* X_fp16,
+                      const void* Wq_packed, const void* W_scales, void* Y_fp16, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  return linear_common(M, N, K, group_size, 6, X_fp16, Wq_packed, W_scales, Y_fp16, workspace,
+                       workspace_bytes, stream);
+}
+
+int flexq_linear_w6a8(int M, int N, int K, int group_size, const void* X_fp16,
+                      const void* Wq_packed, const void* W_scales, void* Y_fp16, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  return linear_common(M, N, K, group_size, 8, X_fp16, Wq_packed, W_scales, Y_fp16, workspace,
+                       workspace_bytes, stream);
 }
 
 int flexq_debug_check_quantizer(unsigned long long* mismatches, unsigned int* first_mismatch) {

@@ -44,6 +44,7 @@
 #include <type_traits>
 
 #include "flexq_ptx.cuh"
+#include "flexq_quant.cuh"
 
 namespace flexq {
 
@@ -56,6 +57,9 @@ struct GemmArgs {
   const uint8_t* wp;       // packed weights, device form
   __half* y;               // [M, N] output (GEMM mode)
   int32_t* p;              // [G, M, N] partials (debug mode)
+  const __half* x;         // [M, K] FP16 activations (fused quantization only)
+  int qmax;                // activation code range Q (fused quantization only)
+  int fq_offset;           // byte offset of the fused quantizer's smem block
   float* ws_part;          // split-K partial tiles [tiles][split][T][128] (split > 1)
   unsigned int* ws_cnt;    // split-K arrival counters [tiles], zero between calls
   unsigned int* status;    // device status word [4]
@@ -220,7 +224,104 @@ __device__ __forceinline__ void unpack_block(uint32_t w0, uint32_t w1, uint32_t 
   out[3] = ((p2 * 4u + p1) * 4u + p0) * 4u;
 }
 
-template <int T, bool PARTIALS>
+// ---------------------------------------------------------------------------
+// Fused activation quantization (FUSEDQ, token tiles of 16 rows): the kernel
+// reads the FP16 activations itself.  Unpack warp q quantizes rows q, q + 4,
+// q + 8, q + 12 of each stage's 256 codes of K -- lane l owns codes
+// 8l .. 8l+7, a group is gs/8 lanes -- by the code rule of the activation
+// quantizer (flexq_quant.cuh), and stores
+//   * the int8 codes into the stage's activation tile, in the layout the TMA
+//     would have written: row r of a 128-code block at r * 128 bytes, its
+//     16-byte chunk c at position c ^ (r % 8) (128-byte swizzle);
+//   * the FP16 group scales into a ring of per-stage scale slots ([8][T],
+//     group within the stage x token), read by the epilogue.
+// Rows past Mt are never written: their codes multiply a zero scale.
+// ---------------------------------------------------------------------------
+constexpr int kQaSlots = 8;           // per-stage activation-scale slots
+constexpr int kQaRowsTogether = 1;    // rows whose arithmetic interleaves
+
+template <int T>
+struct FusedQLayout {
+  static constexpr int kSlotHalves = 8 * T;
+  static constexpr int kBytes = 2 * kQaSlots * 8 + kQaSlots * kSlotHalves * 2;
+};
+
+// FP16 rows m0 + 4r (r < R, below Mt) of codes k0 .. k0+255, 16 bytes per lane.
+template <int R>
+__device__ __forceinline__ void load_act_rows(uint4 (&xv)[R], const __half* __restrict__ xt,
+                                              int Mt, int K, int m0, int k0, int lane) {
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int m = m0 + 4 * r;
+    xv[r] = make_uint4(0u, 0u, 0u, 0u);
+    if (m < Mt)
+      xv[r] = __ldg(reinterpret_cast<const uint4*>(xt + static_cast<size_t>(m) * K + k0) + lane);
+  }
+}
+
+// RG rows m0, m0 + 4, ... at once, by the activation quantizer's route
+// (group_scale_fast, quantize8).
+template <int T, int RG>
+__device__ __forceinline__ void quantize_act_group(const uint4* raw, int Mt, int m0, int lanes,
+                                                   int grp, int qmax, uint8_t* xs,
+                                                   __half* qa_slot, int lane) {
+  const float fq = static_cast<float>(qmax);
+  const float rq = __frcp_rn(fq);
+  const int kb = lane >> 4;                              // 128-code block of the stage
+  const int chunk = (lane & 15) >> 1;                    // 16-byte chunk in the block
+  const int half8 = (lane & 1) * 8;                      // byte offset in the chunk
+  float v[RG][8], amax[RG];
+#pragma unroll
+  for (int r = 0; r < RG; ++r) {
+    const __half2* h2 = reinterpret_cast<const __half2*>(&raw[r]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(h2[i]);
+      v[r][2 * i] = f.x;
+      v[r][2 * i + 1] = f.y;
+    }
+    amax[r] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax[r] = fmaxf(amax[r], fabsf(v[r][i]));
+  }
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+      const float o = __shfl_xor_sync(0xffffffffu, amax[r], off);
+      if (off < lanes) amax[r] = fmaxf(amax[r], o);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < RG; ++r) {
+    const int m = m0 + 4 * r;
+    const __half s16 = group_scale_fast(amax[r], fq, rq);
+    const float sc = __half2float(s16);
+    const uint2 codes = quantize8(v[r], sc, rcp_estimate(sc), qmax);
+    if (m < Mt) {
+      *reinterpret_cast<uint2*>(xs + kb * (T * 128) + m * 128 + ((chunk ^ (m & 7)) << 4) + half8) =
+          codes;
+      if ((lane & (lanes - 1)) == 0) qa_slot[grp * T + m] = s16;
+    }
+  }
+}
+
+// This warp's R rows of one stage (m0 + 4r), RG at a time.
+template <int T, int R, int RG>
+__device__ __forceinline__ void quantize_act_rows(uint4 (&xv)[R], int Mt, int m0, int gs_log2,
+                                                  int qmax, uint8_t* xs, __half* qa_slot,
+                                                  int lane) {
+  static_assert(R % RG == 0, "row groups");
+  const int lanes = (1 << gs_log2) >> 3;                 // lanes per group (4..32)
+  const int grp = (lane * 8) >> gs_log2;                 // group within the stage
+#pragma unroll
+  for (int r = 0; r < R; r += RG) {
+    if (m0 + 4 * r >= Mt) break;                         // uniform across the warp
+    quantize_act_group<T, RG>(&xv[r], Mt, m0 + 4 * r, lanes, grp, qmax, xs, qa_slot, lane);
+  }
+}
+
+template <int T, bool PARTIALS, bool FUSEDQ = false>
 __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     gemm_w6ax_kernel(const __grid_constant__ CUtensorMap tmap_x,
                      const __grid_constant__ CUtensorMap tmap_sa,
@@ -235,6 +336,11 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   uint8_t* w_ring = base + STAGES * Cfg::kXsBytes;          // STAGES * 24576
   uint8_t* sc_ring = w_ring + STAGES * Cfg::kWStageBytes;   // kScSlots slots
   GemmCtrl<T>* ctrl = reinterpret_cast<GemmCtrl<T>*>(base + args.ctrl_offset);
+  // fused quantization: per-stage activation-scale slots and their barriers
+  static_assert(!FUSEDQ || (T == 16 && !PARTIALS && ASLOTS == STAGES), "fused quantization");
+  uint64_t* qa_full = reinterpret_cast<uint64_t*>(base + args.fq_offset);   // 4 unpack warps
+  uint64_t* qa_empty = qa_full + kQaSlots;                                   // epilogue warps
+  __half* qa_ring = reinterpret_cast<__half*>(qa_empty + kQaSlots);          // [slot][8][T]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -292,12 +398,23 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       mbar_init(&ctrl->s_empty[s], Cfg::kEpiWarps);
     }
     mbar_init(&ctrl->done, 1);
+    if (FUSEDQ) {
+      for (int s = 0; s < kQaSlots; ++s) {
+        mbar_init(&qa_full[s], 4);
+        mbar_init(&qa_empty[s], Cfg::kEpiWarps);
+      }
+    }
     fence_barrier_init();
-    prefetch_tensormap(&tmap_x);
+    if (!FUSEDQ) prefetch_tensormap(&tmap_x);
     if (!PARTIALS) {
-      prefetch_tensormap(&tmap_sa);
+      if (!FUSEDQ) prefetch_tensormap(&tmap_sa);
       prefetch_tensormap(&tmap_sw);
     }
+  }
+  if (FUSEDQ) {
+    // tokens past M keep a zero scale in every slot
+    for (int i = threadIdx.x; i < kQaSlots * 8 * T / 8; i += blockDim.x)
+      reinterpret_cast<uint4*>(qa_ring)[i] = make_uint4(0u, 0u, 0u, 0u);
   }
   if (warp == 1) tmem_alloc(&ctrl->tmem_base, Cfg::kTmemCols);
   tc_fence_before();
@@ -324,9 +441,13 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       // requested before waiting for the kernels this one depends on (whose
       // outputs may be this kernel's activations and their scales).
       const int n_pre = nst < STAGES ? nst : STAGES;
+      // with fused quantization the stage's copy is the weights alone, and
+      // the scale slots receive the weight scales only
+      constexpr uint32_t kStageTx = FUSEDQ ? Cfg::kWStageBytes : Cfg::kStageBytes;
+      constexpr uint32_t kScTx = FUSEDQ ? Cfg::kScSlotBytes - Cfg::kScSaBytes : Cfg::kScSlotBytes;
       for (int i = 0; i < n_pre; ++i) {
         if (args.stall && i == 0) continue;
-        mbar_arrive_expect_tx(&ctrl->full[i], Cfg::kStageBytes);
+        mbar_arrive_expect_tx(&ctrl->full[i], kStageTx);
         bulk_load(w_ring + i * Cfg::kWStageBytes,
                   args.wp + (static_cast<size_t>(nt) * KB + kb0 + 2 * i) * kWTileBytes,
                   Cfg::kWStageBytes, &ctrl->full[i]);
@@ -343,8 +464,8 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
             break;
           }
           uint8_t* dst = sc_ring + slot * Cfg::kScSlotBytes;
-          mbar_arrive_expect_tx(&ctrl->s_full[slot], Cfg::kScSlotBytes);
-          tma_load_2d(dst, &tmap_sa, &ctrl->s_full[slot], mt * T, g0 + 8 * o);
+          mbar_arrive_expect_tx(&ctrl->s_full[slot], kScTx);
+          if (!FUSEDQ) tma_load_2d(dst, &tmap_sa, &ctrl->s_full[slot], mt * T, g0 + 8 * o);
           tma_load_2d(dst + Cfg::kScSaBytes, &tmap_sw, &ctrl->s_full[slot], nt * kTileRows,
                       g0 + 8 * o);
           sc_issued |= 1u << slot;
@@ -363,14 +484,16 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         const int kb = kb0 + 2 * i;
         uint8_t* xs = xs_ring + s * Cfg::kXsBytes;
         if (i >= n_pre) {
-          mbar_arrive_expect_tx(&ctrl->full[s], Cfg::kStageBytes);
+          mbar_arrive_expect_tx(&ctrl->full[s], kStageTx);
           // tiles (nt, kb) and (nt, kb + 1) are adjacent in the device form
           bulk_load(w_ring + s * Cfg::kWStageBytes,
                     args.wp + (static_cast<size_t>(nt) * KB + kb) * kWTileBytes,
                     Cfg::kWStageBytes, &ctrl->full[s]);
         }
-        tma_load_2d(xs, &tmap_x, &ctrl->full[s], kb * kKBlock, mt * T);
-        tma_load_2d(xs + Cfg::kXsHalf, &tmap_x, &ctrl->full[s], (kb + 1) * kKBlock, mt * T);
+        if (!FUSEDQ) {
+          tma_load_2d(xs, &tmap_x, &ctrl->full[s], kb * kKBlock, mt * T);
+          tma_load_2d(xs + Cfg::kXsHalf, &tmap_x, &ctrl->full[s], (kb + 1) * kKBlock, mt * T);
+        }
         issued |= 1u << s;
         parity = (parity & ~(1u << s)) | (static_cast<uint32_t>((i / STAGES) & 1) << s);
       }
@@ -474,11 +597,47 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     FLEXQ_ROLE_CLOCK;
     RingPos<STAGES> st;
     RingPos<ASLOTS> as;
+    // fused quantization: this warp's activation rows, loaded during the
+    // previous stage
+    constexpr int R = FUSEDQ ? T / 4 : 1;
+    uint4 xv[R];
+    RingPos<kQaSlots> qp;
+    const __half* xt = args.x + static_cast<size_t>(mt) * T * K;   // the token tile's rows
+    const int Mt = min(T, M - mt * T);
+    if constexpr (FUSEDQ) {
+      grid_wait_dependencies();                   // the activations may come from the previous kernel
+      load_act_rows<R>(xv, xt, Mt, K, q, kb0 * kKBlock, lane);
+    }
     for (int i = 0; i < nst; ++i) {
-      if (!FLEXQ_WAIT(warp_wait(&ctrl->full[st.idx], st.phase, lim)) ||
-          !FLEXQ_WAIT(warp_wait(&ctrl->a_empty[as.idx], as.phase ^ 1u, lim))) {
-        if (lane == 0) record_status(args.status, kStatusTimeout, 2);
-        break;
+      if constexpr (FUSEDQ) {
+        // the stage's activation tile is free once its A slot is: the same
+        // MMA commit releases both (as many A slots as stages)
+        if (!FLEXQ_WAIT(warp_wait(&ctrl->a_empty[as.idx], as.phase ^ 1u, lim)) ||
+            !FLEXQ_WAIT(warp_wait(&qa_empty[qp.idx], qp.phase ^ 1u, lim))) {
+          if (lane == 0) record_status(args.status, kStatusTimeout, 2);
+          break;
+        }
+        uint4 cur[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) cur[r] = xv[r];
+        quantize_act_rows<T, R, kQaRowsTogether>(cur, Mt, q, gs_log2, args.qmax,
+                                                 xs_ring + st.idx * Cfg::kXsBytes,
+                                                 qa_ring + qp.idx * FusedQLayout<T>::kSlotHalves,
+                                                 lane);
+        fence_proxy_async_smem();                 // codes -> the MMA's operand reads
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qa_full[qp.idx]);
+        qp.next();
+        if (!FLEXQ_WAIT(warp_wait(&ctrl->full[st.idx], st.phase, lim))) {
+          if (lane == 0) record_status(args.status, kStatusTimeout, 2);
+          break;
+        }
+      } else {
+        if (!FLEXQ_WAIT(warp_wait(&ctrl->full[st.idx], st.phase, lim)) ||
+            !FLEXQ_WAIT(warp_wait(&ctrl->a_empty[as.idx], as.phase ^ 1u, lim))) {
+          if (lane == 0) record_status(args.status, kStatusTimeout, 2);
+          break;
+        }
       }
       tc_fence_after();                           // the MMAs that read slot a are done
       // this row's packed bytes: tile t, chunk j at t*12288 + (j*128 + row)*16
@@ -505,6 +664,9 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->a_full[as.idx]);
+      // fused quantization: the next stage's rows, requested once this
+      // stage's weights are out of the registers
+      if (FUSEDQ && i + 1 < nst) load_act_rows<R>(xv, xt, Mt, K, q, (kb0 + 2 * i + 2) * kKBlock, lane);
       st.next();
       as.next();
     }
@@ -525,6 +687,8 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     // ring slot and its release happen once per octet
     RingPos<NB> pb;
     RingPos<Cfg::kScSlots> sp;                       // scale-ring slot of the octet
+    RingPos<kQaSlots> qp;                            // fused quantization: stage scale slot
+    const int G_st = Cfg::kKStage >> gs_log2;        // groups per stage
     bool failed = false;
     for (int lo = 0; lo < ngroups && !failed; lo += 8) {
       const uint8_t* sc = sc_ring + sp.idx * Cfg::kScSlotBytes;
@@ -534,20 +698,38 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
           if (lane == 0) record_status(args.status, kStatusTimeout, 5);
           break;
         }
-        // this warp's tokens of the octet, FP16 -> FP32, into its own buffer
-        const __half* sa_h = reinterpret_cast<const __half*>(sc);
+        if (!FUSEDQ) {
+          // this warp's tokens of the octet, FP16 -> FP32, into its own buffer
+          const __half* sa_h = reinterpret_cast<const __half*>(sc);
 #pragma unroll
-        for (int idx = lane; idx < 8 * Cfg::kCols; idx += 32) {
-          const int gg = idx / Cfg::kCols, j = idx - gg * Cfg::kCols;
-          ctrl->sa[e][gg][j] = __half2float(sa_h[gg * T + col0 + j]);
+          for (int idx = lane; idx < 8 * Cfg::kCols; idx += 32) {
+            const int gg = idx / Cfg::kCols, j = idx - gg * Cfg::kCols;
+            ctrl->sa[e][gg][j] = __half2float(sa_h[gg * T + col0 + j]);
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
 #pragma unroll
       for (int gi = 0; gi < 8; ++gi) {
       const int lg = lo + gi;
       if (lg >= ngroups) break;
       const int g = g0 + lg;
+      if (FUSEDQ && (lg & (G_st - 1)) == 0) {
+        // first group of a stage: its activation scales, from the unpack warps
+        if (!FLEXQ_WAIT(warp_wait(&qa_full[qp.idx], qp.phase, lim))) {
+          if (lane == 0) record_status(args.status, kStatusTimeout, 6);
+          failed = true;
+          break;
+        }
+        const __half* qa = qa_ring + qp.idx * FusedQLayout<T>::kSlotHalves;
+        for (int idx = lane; idx < G_st * Cfg::kCols; idx += 32) {
+          const int j = idx / Cfg::kCols, t = idx - j * Cfg::kCols;
+          ctrl->sa[e][gi + j][t] = __half2float(qa[j * T + col0 + t]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qa_empty[qp.idx]);
+        qp.next();
+      }
       float swn = 0.0f;
       if (!PARTIALS) swn = __half2float(sw_h[gi * kTileRows + row]) * 0.25f;
       const float* sa_w = ctrl->sa[e][gi];

@@ -62,6 +62,66 @@ __device__ __forceinline__ int quant_code(float x, float s, float rs, int qmax) 
   return s == 0.0f ? 0 : quant_code_fast(x, s, rs, qmax);
 }
 
+// ---- the route the quantizers take (division-free, no conversion unit) ----
+// s32 = RN(a / Q) for a finite FP16 value a >= 0 and Q in {31, 127}, given
+// rq = RN(1 / Q): the estimate q0 = RN(a * rq) is corrected once by its
+// exact residual a - q0 * Q (q0 has 24 significant bits, Q at most 7, and
+// the residual is far below a).  The result equals the IEEE division for
+// every FP16 a and both Q (flexq_debug_check_quantizer checks all of them).
+__device__ __forceinline__ float div_by_q(float a, float fq, float rq) {
+  const float q0 = __fmul_rn(a, rq);
+  const float r = __fmaf_rn(-q0, fq, a);
+  return __fmaf_rn(r, rq, q0);
+}
+
+__device__ __forceinline__ __half group_scale_fast(float amax, float fq, float rq) {
+  return __float2half_rn(div_by_q(amax, fq, rq));
+}
+
+// Reciprocal estimate of a positive FP32 value converted from FP16 (a normal
+// FP32 number): one approximate reciprocal, within about one ulp.  Both code
+// routes only need x * rs to land within 2^-14 of x / s (quant_code_fast).
+__device__ __forceinline__ float rcp_estimate(float s) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+  return r;
+}
+
+// Common route for one value whose group has a normal FP16 scale s, so that
+// |x / s| < Q + 1/2 (the stored scale is within 2^-11 of amax / Q): with
+// t = RN(x * rs + 1.5 * 2^23), the low mantissa bits of t hold the integer
+// k = rint(x * rs), so the low byte of t's bit pattern is k's two's
+// complement byte.  k equals round_half_even(x / s) unless x / s is exactly a
+// half-integer, which shows as an exact residual |x - k * s| = s / 2 and is
+// flagged in `tie` for the full rule.  No clamp is needed below Q + 1/2.
+constexpr float kRoundMagic = 12582912.0f;            // 1.5 * 2^23
+
+__device__ __forceinline__ uint32_t code_bits_common(float x, float s, float rs, float half_s,
+                                                     bool& tie) {
+  const float t = __fmaf_rn(x, rs, kRoundMagic);
+  const float k = __fsub_rn(t, kRoundMagic);
+  tie |= fabsf(__fmaf_rn(-k, s, x)) == half_s;
+  return __float_as_uint(t);
+}
+
+// Eight consecutive values of one group -> their codes' low bytes in order,
+// packed in two words.  Values whose group scale is subnormal or zero, and
+// groups of this lane that meet a tie, take the full rule (quant_code).
+__device__ __forceinline__ uint2 quantize8(const float (&v)[8], float sc, float rs, int qmax) {
+  const float half_s = 0.5f * sc;
+  bool exact = !(sc >= 6.103515625e-05f);             // subnormal or zero scale
+  uint32_t b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) b[i] = code_bits_common(v[i], sc, rs, half_s, exact);
+  if (exact) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b[i] = static_cast<uint32_t>(quant_code(v[i], sc, rs, qmax));
+  }
+  const uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+  return make_uint2(lo, hi);
+}
+
 // --------------------------------------------------------------------------
 // Activation quantization: each thread owns 8 consecutive values (one 16-byte
 // load); a group is gs/8 consecutive lanes (4..32), reduced with shuffles.
@@ -86,6 +146,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(
   const int c = t % chunks_per_row;
   const int row0 = t / chunks_per_row;
   const float fq = static_cast<float>(qmax);
+  const float rq = __frcp_rn(fq);
   const int steps = (M + rows_per_step - 1) / rows_per_step;
   for (int st0 = 0; st0 < steps; st0 += U) {
     uint4 raw[U];
@@ -114,36 +175,11 @@ __global__ void __launch_bounds__(256) quant_act_kernel(
 #pragma unroll
       for (int off = 1; off < LANES; off <<= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      const __half s16 = group_scale(amax, fq);
+      const __half s16 = group_scale_fast(amax, fq, rq);
       const float sc = __half2float(s16);
-      const float rs = sc == 0.0f ? 0.0f : __frcp_rn(sc);
-      // Common path: rint(x * rs) is the code unless x/s is exactly a
-      // half-integer (see quant_code_fast), and a normal FP16 scale
-      // (>= 2^-14, rounded from absmax/Q with relative error <= 2^-11) keeps
-      // every |x/s| below Q + 1/2, so no clamp is needed.  A tie shows as an
-      // exact residual of s/2.  Warps that meet a tie or a subnormal or zero
-      // scale take the full rule for all their values.
-      const float h = 0.5f * sc;
-      float kf[8];
-      bool exact_path = !(sc >= 6.103515625e-05f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        kf[i] = rintf(v[i] * rs);
-        exact_path |= fabsf(fmaf(-kf[i], sc, v[i])) == h;
-      }
-      int q[8];
-      if (__any_sync(0xffffffffu, exact_path)) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = quant_code(v[i], sc, rs, qmax);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = __float2int_rn(kf[i]);
-      }
-      // low bytes of the codes, in order, two permutes per four codes
-      const uint32_t lo = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
-      const uint32_t hi = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
+      const uint2 codes = quantize8(v, sc, rcp_estimate(sc), qmax);
       if (row < M) {
-        Xq[static_cast<long long>(row) * chunks_per_row + c] = make_uint2(lo, hi);
+        Xq[static_cast<long long>(row) * chunks_per_row + c] = codes;
         if ((c % LANES) == 0) Xs[static_cast<long long>(c / LANES) * ld_scales + row] = s16;
       }
     }
@@ -248,9 +284,13 @@ __global__ void __launch_bounds__(256) weight_pack_kernel(
 
 // --------------------------------------------------------------------------
 // Test hook: for FP16 scale patterns [s_first, s_first + n_s) (positive,
-// finite) against every finite FP16 value x, counts the (x, s) pairs where
-// quant_code_fast differs from quant_code_div, for Q = 31 and Q = 127, and
-// records the first mismatch.  One thread per (x, s) pair.
+// finite) against every finite FP16 value x, for Q = 31 and Q = 127, counts
+// the (x, s) pairs where a route of the quantizers differs from
+// quant_code_div: quant_code_fast with either reciprocal, and the common
+// route wherever a group can take it (its tie flag must be raised exactly at
+// the half-integer quotients); with the first scale pattern, also every
+// non-negative FP16 x as a group maximum through group_scale_fast.  Records
+// the first mismatch.  One thread per (x, s) pair.
 // --------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) check_quantizer_kernel(unsigned s_first, unsigned n_s,
                                                               unsigned long long* mismatches,
@@ -263,10 +303,27 @@ __global__ void __launch_bounds__(256) check_quantizer_kernel(unsigned s_first, 
   const float x = __half2float(__ushort_as_half(static_cast<unsigned short>(xb)));
   const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(sb)));
   const float rs = __frcp_rn(s);
+  const float rse = rcp_estimate(s);
   const int qs[2] = {31, 127};
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    if (quant_code_fast(x, s, rs, qs[i]) != quant_code_div(x, s, qs[i])) {
+    const int want = quant_code_div(x, s, qs[i]);
+    // the full rule, with the correctly rounded and with the estimated
+    // reciprocal
+    bool bad = quant_code_fast(x, s, rs, qs[i]) != want || quant_code_fast(x, s, rse, qs[i]) != want;
+    // the common route, wherever a group can use it: a normal scale and
+    // |x / s| <= Q + 1/2 (a tie there must be flagged)
+    if (s >= 6.103515625e-05f && fabsf(x) <= (static_cast<float>(qs[i]) + 0.5f) * s) {
+      bool tie = false;
+      const uint32_t t = code_bits_common(x, s, rse, 0.5f * s, tie);
+      // (a flagged pair takes the full rule, checked above)
+      if (!tie) bad |= static_cast<int>(static_cast<int8_t>(t & 0xFFu)) != want;
+    }
+    // the scale: every FP16 value as a group's absolute maximum
+    if (sb == 1u && !(xb & 0x8000u))
+      bad |= __half_as_ushort(group_scale_fast(x, static_cast<float>(qs[i]), __frcp_rn(static_cast<float>(qs[i])))) !=
+             __half_as_ushort(group_scale(x, static_cast<float>(qs[i])));
+    if (bad) {
       if (atomicAdd(mismatches, 1ull) == 0ull) {
         first[0] = xb;
         first[1] = sb;

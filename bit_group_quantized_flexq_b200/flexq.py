@@ -56,6 +56,11 @@ def lib():
             "flexq_gemm_w6a8": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p,
                                         c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                         c_void_p]),
+            "flexq_linear_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
+            "flexq_linear_w6a6": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p,
+                                          c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+            "flexq_linear_w6a8": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p,
+                                          c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
             "flexq_gemm_static_scratch": (c_int, [c_int, c_int, c_int, c_int, c_int, c_void_p,
                                                   c_void_p, c_void_p, c_void_p, c_void_p,
                                                   c_void_p]),
@@ -67,6 +72,8 @@ def lib():
                                         ctypes.POINTER(c_int), ctypes.POINTER(c_int),
                                         ctypes.POINTER(c_int)]),
             "flexq_debug_force_plan": (c_int, [c_int, c_int]),
+            "flexq_linear_launches": (c_int, [c_int, c_int, c_int, c_int]),
+            "flexq_debug_force_linear_route": (c_int, [c_int]),
             "flexq_set_wait_limit_ns": (c_int, [ctypes.c_uint64]),
             "flexq_debug_inject_stall": (c_int, [c_int]),
             "flexq_get_device_status": (c_int, [c_void_p]),
@@ -220,6 +227,51 @@ def gemm(xq, xs, wp, ws, N, group_size, act_bits=6, out=None, workspace_buf=None
     return out
 
 
+def linear_workspace_bytes(M, N, K, group_size):
+    return int(lib().flexq_linear_workspace_bytes(M, N, K, group_size))
+
+
+def linear_launches(M, N, K, group_size):
+    """1 where linear() quantizes inside the GEMM (one launch), 2 where it runs
+    the quantizer and then the GEMM, 0 for unsupported shapes."""
+    return int(lib().flexq_linear_launches(M, N, K, group_size))
+
+
+def force_linear_route(route=0):
+    """Test hook: 0 by shape, 1 quantization inside the GEMM wherever the
+    plan's token tile is 16 rows, 2 always the separate quantizer."""
+    _check(lib().flexq_debug_force_linear_route(route))
+
+
+def linear(x, wp, ws, N, group_size, act_bits=6, out=None, workspace_buf=None):
+    """Y [M, N] FP16 of a quantized linear layer from FP16 activations x
+    [M, K]: the activations are quantized to act_bits (6 or 8) by the rule of
+    quantize_act, then multiplied with the packed 6-bit weights.  Batches of
+    at most 2 tokens quantize inside the GEMM (one launch; linear_launches).
+
+    workspace_buf: a zero-filled uint8 device tensor of at least
+    linear_workspace_bytes(M, N, K, gs) bytes; by default a per-device shared
+    one."""
+    _need(x, "x", torch.float16)
+    M, K = x.shape
+    _need(wp, "wp", torch.uint8, (weight_packed_bytes(N, K, group_size),))
+    _need(ws, "ws", torch.float16, (K // group_size, N))
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.float16, device=x.device)
+    _need(out, "out", torch.float16, (M, N))
+    if workspace_buf is None:
+        need = linear_workspace_bytes(M, N, K, group_size)
+        workspace_buf = workspace(x.device, need) if need else None
+    if workspace_buf is None or workspace_buf.numel() == 0:
+        wsp, wsn = ctypes.c_void_p(0), 0
+    else:
+        _need(workspace_buf, "workspace", torch.uint8)
+        wsp, wsn = _ptr(workspace_buf), workspace_buf.numel()
+    fn = {6: lib().flexq_linear_w6a6, 8: lib().flexq_linear_w6a8}[act_bits]
+    _check(fn(M, N, K, group_size, _ptr(x), _ptr(wp), _ptr(ws), _ptr(out), wsp, wsn, _stream(x)))
+    return out
+
+
 def gemm_static_scratch(xq, xs, wp, ws, N, group_size, act_bits=6, out=None):
     """The GEMM through flexq_gemm_static_scratch: no workspace argument and
     no device allocation by the library (the split-K scratch is a fixed array
@@ -257,12 +309,6 @@ def debug_group_partials(xq, wp, N, group_size, out=None):
     _check(lib().flexq_debug_group_partials(M, N, K, group_size, _ptr(xq), _ptr(wp), _ptr(out),
                                             _stream(xq)))
     return out
-
-
-def linear(x, wp, ws, N, group_size, act_bits=6, xq_out=None, y_out=None):
-    """One linear layer on FP16 activations: quantize X, then the group GEMM."""
-    xq, xs = quantize_act(x, group_size, act_bits, out=xq_out)
-    return gemm(xq, xs, wp, ws, N, group_size, act_bits, out=y_out)
 
 
 def plan(M, N, K, group_size):

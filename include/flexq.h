@@ -168,6 +168,60 @@ int flexq_gemm_w6a8(int M, int N, int K, int group_size, const int8_t* Xq,
                     size_t workspace_bytes, void* stream);
 
 /*
+ * flexq_linear_workspace_bytes -- device workspace the linear entry points
+ * need for a shape.  Shapes that quantize inside the GEMM (see
+ * flexq_linear_launches) need exactly flexq_gemm_workspace_bytes; the others
+ * also hold the quantized activations: 4096 bytes of arrival counters (or the
+ * GEMM workspace if larger), then the [M, K] int8 codes and the FP16 scales
+ * (G * flexq_act_scales_ld(M) values), each starting on a 256-byte boundary.
+ * Pure host computation; 0 for unsupported shapes and M <= 0.
+ */
+size_t flexq_linear_workspace_bytes(int M, int N, int K, int group_size);
+
+/*
+ * flexq_linear_launches -- kernel launches of one linear call for a shape:
+ * 1 where the activations are quantized inside the GEMM (batches of at most
+ * 2 tokens on 16-token tiles, the sizes where that is not slower than a
+ * separate quantizer), 2 otherwise (quantizer, GEMM).  0 for unsupported
+ * shapes and M <= 0.  Pure host computation.
+ */
+int flexq_linear_launches(int M, int N, int K, int group_size);
+
+/*
+ * flexq_linear_w6a6 / flexq_linear_w6a8 -- a quantized linear layer from
+ * FP16 activations: Y = dequant(quant_a(X)) . dequant(Wq)^T with quant_a the
+ * 6-bit (w6a6) or 8-bit (w6a8) activation quantizer of flexq_quantize_act.
+ * Passage: activations quantized per group at run time and multiplied with
+ * the 6-bit weights, dequantization fused into the GEMM (arXiv abstract;
+ * blog, "Fine-Grained Quantization and Layer Sensitivity" and "Bridging
+ * Software and Hardware with BTC").
+ *
+ *   X_fp16           [M, K] FP16 activations, finite values, 16-byte aligned.
+ *   Wq_packed,       as for flexq_gemm_w6a6.
+ *   W_scales
+ *   Y_fp16           out, [M, N] FP16.
+ *   workspace,       device scratch of flexq_linear_workspace_bytes(M, N, K,
+ *   workspace_bytes  gs) bytes or more, owned by the caller, 16-byte
+ *                    aligned, zero-filled before its first use (completed
+ *                    calls leave its counters zero again).  Where the
+ *                    quantization runs inside the GEMM, NULL with 0 bytes
+ *                    runs without a K split, as for the GEMM; elsewhere the
+ *                    workspace is required (FLEXQ_ERR_INVALID_ARG).
+ * Batches of at most 2 tokens quantize the activations inside the GEMM
+ * kernel (one launch, no quantized copy in device memory); larger ones launch
+ * the activation quantizer into the workspace and then the GEMM.  Both routes
+ * compute the same codes and scales as flexq_quantize_act, and the result is
+ * bit-identical to flexq_quantize_act followed by flexq_gemm_w6a6/w6a8 under
+ * the same plan.
+ */
+int flexq_linear_w6a6(int M, int N, int K, int group_size, const void* X_fp16,
+                      const void* Wq_packed, const void* W_scales, void* Y_fp16,
+                      void* workspace, size_t workspace_bytes, void* stream);
+int flexq_linear_w6a8(int M, int N, int K, int group_size, const void* X_fp16,
+                      const void* Wq_packed, const void* W_scales, void* Y_fp16,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * flexq_gemm_static_scratch -- the GEMM of flexq_gemm_w6a6 (act_bits 6) or
  * flexq_gemm_w6a8 (act_bits 8) for callers that cannot allocate device
  * memory when they call it: an engine plugin whose enqueue step may not
@@ -203,6 +257,14 @@ int flexq_gemm_static_scratch(int M, int N, int K, int group_size, int act_bits,
  */
 int flexq_debug_check_quantizer(unsigned long long* mismatches,
                                 unsigned int* first_mismatch);
+
+/*
+ * flexq_debug_force_linear_route -- test hook: 0 picks the linear route by
+ * shape (flexq_linear_launches), 1 quantizes inside the GEMM whenever the
+ * plan's token tile is 16 rows, 2 always runs the separate quantizer.
+ * Process-wide; FLEXQ_ERR_INVALID_ARG for other values.
+ */
+int flexq_debug_force_linear_route(int route);
 
 /*
  * flexq_debug_group_partials -- exports the per-group int32 partials of the

@@ -125,3 +125,36 @@ def test_workspace_size_follows_the_plan(L):
         assert flexq.gemm_workspace_bytes(M, N, K, 128) == want
     assert flexq.gemm_workspace_bytes(0, 4096, 4096, 128) == 0
     assert flexq.gemm_workspace_bytes(4, 200, 4096, 128) == 0
+
+
+def test_linear_validation_before_any_launch(L):
+    f = L.flexq_linear_w6a6
+    # bad bit width (the w6a6/w6a8 wrappers fix it), shapes, pointers
+    assert f(4, 200, 256, 128, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
+    assert f(4, 256, 256, 48, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
+    assert f(4, 256, 256, 128, NULL, FAKE, FAKE, FAKE, NULL, 0, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert b"X_fp16" in L.flexq_last_error_message()
+    assert f(4, 256, 256, 128, MISALIGNED, FAKE, FAKE, FAKE, NULL, 0, NULL) == flexq.FLEXQ_ERR_MISALIGNED
+    assert L.flexq_linear_w6a8(-1, 256, 256, 128, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == \
+        flexq.FLEXQ_ERR_INVALID_ARG
+    assert f(0, 256, 256, 128, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == flexq.FLEXQ_OK   # empty batch
+
+
+def test_linear_workspace_layout(L):
+    # batches of at most 2 tokens quantize inside the GEMM: the GEMM's workspace alone
+    for M, N, K in [(1, 4096, 4096), (2, 11008, 4096), (1, 384, 1024)]:
+        assert flexq.linear_launches(M, N, K, 128) == 1
+        assert flexq.linear_workspace_bytes(M, N, K, 128) == flexq.gemm_workspace_bytes(M, N, K, 128)
+    # the others add the codes and the scales after the GEMM region
+    for M, N, K, gs in [(3, 384, 1024, 128), (16, 11008, 4096, 128), (17, 4096, 4096, 128),
+                        (256, 4096, 11008, 64), (2048, 4096, 4096, 128)]:
+        assert flexq.linear_launches(M, N, K, gs) == 2
+        head = max(flexq.gemm_workspace_bytes(M, N, K, gs), 4096)
+        xq_off = (head + 255) // 256 * 256
+        xs_off = (xq_off + M * K + 255) // 256 * 256
+        want = xs_off + (K // gs) * flexq.act_scales_ld(M) * 2
+        assert flexq.linear_workspace_bytes(M, N, K, gs) == want
+    assert flexq.linear_workspace_bytes(0, 4096, 4096, 128) == 0
+    assert flexq.linear_workspace_bytes(4, 200, 4096, 128) == 0
+    assert flexq.linear_launches(0, 4096, 4096, 128) == 0
+    assert L.flexq_debug_force_linear_route(3) == flexq.FLEXQ_ERR_INVALID_ARG
