@@ -475,6 +475,7 @@ def run_flexq(args, rank, world):
     if args.diag and rank == 0:
         result["int8_library_context"] = int8_library_context(W, device, dominant_m)
         result["act_quant"] = act_quant_diagnostics(device, hbm)
+        result["mixed_stack"] = stack_diagnostics(device, hbm, int8_peak)
     if args.e2e:
         result["e2e"] = run_e2e(W, args, device, world)
     if rank == 0 and world == 1 and args.cpu_baseline:
@@ -592,6 +593,40 @@ def act_quant_diagnostics(device, hbm_gbs, K=8192, ms=(1, 2048, 16384), reps=20)
         out.append({"M": M, "K": K, "us": round(us, 2), "GB/s": round(gbs, 1),
                     "bound": "hbm", "frac": round(gbs / hbm_gbs, 4)})
     return out
+
+
+def stack_diagnostics(device, hbm_gbs, int8_peak_tops, ms=(1, 16, 512, 8192)):
+    """The mixed W6A6/W6A8 layer stack (stack.LayerStack) on one LLaMA-2-70B
+    block (q, k, v, o, gate, up, down; 8-bit activations for down), seeded
+    synthetic weights drawn on the device: per M, the device time of one
+    block forward from FP16 activations (CUDA graph of a few forwards), with
+    the HBM roofline for M <= 16 and the int8 roofline above."""
+    import torch
+    from bit_group_quantized_flexq_b200 import flexq, inputs, stack
+    st = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED, device=device)
+    stream = torch.cuda.Stream(device)
+    rows = []
+    for M in ms:
+        acts = {site: inputs.activations(M, K, outlier_frac=0.005, outlier_scale=50.0,
+                                         seed=inputs.layer_seed("70b-x", M, site)).to(device)
+                for site, K in st.sites().items()}
+        out = {name: torch.empty(M, N, dtype=torch.float16, device=device)
+               for name, N, K, _ in st.layers}
+        reps = 2 if M >= 4096 else 5
+        us = _graph_time_us(lambda: st.forward(acts, out), device, stream, reps)
+        flops = sum(2.0 * M * N * K for _, N, K, _ in st.layers)
+        nbytes = sum(linear_bytes(M, N, K, st.gs) for _, N, K, _ in st.layers)
+        bound = "hbm" if M <= 16 else "tensor"
+        gbs = nbytes / (us * 1e-6) / 1e9
+        tops = flops / (us * 1e-6) / 1e12
+        rows.append({"M": M, "us": round(us, 2), "TOPS": round(tops, 2), "GB/s": round(gbs, 1),
+                     "bound": bound,
+                     "frac": round(gbs / hbm_gbs if bound == "hbm" else tops / int8_peak_tops, 4),
+                     "launches": st.launches(M)})
+        del acts, out
+    return {"block": "LLaMA-2-70B (q, k, v, o, gate, up, down)",
+            "act_bits": st.bits, "group_size": st.gs,
+            "packed_MB": round(st.packed_bytes() / 1e6, 1), "by_m": rows}
 
 
 def int8_library_context(W, device, M, reps=20):

@@ -388,19 +388,22 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
 
 // ------------------------------------------------------- linear layers --
 // A linear layer from FP16 activations: quantize them (bits 6 or 8), then the
-// group GEMM.  Batches of at most kFusedMaxM tokens (on 16-token tiles)
-// quantize inside the GEMM (one launch): there the in-kernel quantization,
-// whose rows each unpack warp takes one after another, costs no more than a
-// separate quantizer launch ahead of the GEMM; larger batches run the
-// activation quantizer first, its codes and scales in the caller's workspace
-// after the GEMM's region, whose arrival counters keep their fixed place at
-// the start.
-constexpr int kFusedMaxM = 2;
-
-bool linear_fused(const Plan& p, int M) {
+// group GEMM, in one of two routes.  Inside the GEMM (16-token tiles, one
+// launch) the quantization saves the separate quantizer's launch and its
+// dependency (about 1.4 us per layer) but lengthens every pipeline stage of
+// the unpack warps, by more the more tokens there are; it is taken where
+// each CTA streams few stages: at most 4 stages of K for up to 4 tokens, at
+// most 2 for up to 8 tokens (measured per layer, weights cold: 4096^2 and
+// 1024x8192 layers gain 8-14 % at one token, layers with 6 stages per CTA
+// lose 2-3 %).  Otherwise the activation quantizer runs first, its codes
+// and scales in the caller's workspace after the GEMM's region, whose
+// arrival counters keep their fixed place at the start.
+bool linear_fused(const Plan& p, int M, int K) {
   const int route = g_force_linear_route.load();
   if (p.T != 16) return false;
-  return route == 1 || (route == 0 && M <= kFusedMaxM);
+  if (route != 0) return route == 1;
+  const int stages = (K / 256 + p.split - 1) / p.split;     // per CTA
+  return (M <= 4 && stages <= 4) || (M <= 8 && stages <= 2);
 }
 
 struct LinearLayout {
@@ -412,7 +415,7 @@ struct LinearLayout {
 
 LinearLayout linear_layout(const Plan& p, int M, int N, int K, int gs) {
   LinearLayout L = {};
-  L.fused = linear_fused(p, M);
+  L.fused = linear_fused(p, M, K);
   L.gemm_bytes = workspace_bytes_for(p, M, N);
   if (L.fused) {
     L.total = L.gemm_bytes;

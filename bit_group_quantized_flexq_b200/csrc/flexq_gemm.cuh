@@ -198,11 +198,14 @@ __device__ __forceinline__ void record_status(unsigned int* status, int code,
   }
 }
 
-// Lane 0 waits (the other lanes park at the warp barrier instead of polling
-// the mbarrier); the warp agrees on the outcome.  The warp barrier orders the
-// waiting lane's acquire before every lane's subsequent reads.
+// Otherwise lane 0 waits (the other lanes park at the warp barrier instead of
+// polling the mbarrier); the warp agrees on the outcome.  The warp barrier
+// orders the waiting lane's acquire before every lane's subsequent reads.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
                                           uint64_t limit) {
+  // fast path: the phase is usually complete already; every lane probes it
+  // (each probe acquires for its own lane) and one vote settles it
+  if (__all_sync(0xffffffffu, mbar_test_wait(smem_u32(bar), parity))) return true;
   bool ok = true;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, limit);
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -226,8 +229,9 @@ __device__ __forceinline__ void unpack_block(uint32_t w0, uint32_t w1, uint32_t 
 
 // ---------------------------------------------------------------------------
 // Fused activation quantization (FUSEDQ, token tiles of 16 rows): the kernel
-// reads the FP16 activations itself.  Unpack warp q quantizes rows q, q + 4,
-// q + 8, q + 12 of each stage's 256 codes of K -- lane l owns codes
+// reads the FP16 activations itself.  At stage i unpack warp q quantizes rows
+// m0, m0 + 4, ... with m0 = (q - i * Mt) mod 4 (fq_row0) of the stage's 256
+// codes of K -- lane l owns codes
 // 8l .. 8l+7, a group is gs/8 lanes -- by the code rule of the activation
 // quantizer (flexq_quant.cuh), and stores
 //   * the int8 codes into the stage's activation tile, in the layout the TMA
@@ -245,6 +249,14 @@ struct FusedQLayout {
   static constexpr int kSlotHalves = 8 * T;
   static constexpr int kBytes = 2 * kQaSlots * 8 + kQaSlots * kSlotHalves * 2;
 };
+
+// First row of unpack warp q at stage i: the stage's (stage, row) pairs are
+// dealt to the four warps in turn, so a batch of one or two rows spreads its
+// quantization over all four warps across consecutive stages instead of
+// loading one warp with every stage.
+__device__ __forceinline__ int fq_row0(int q, int i, int Mt) {
+  return (q - (i * Mt) % 4 + 4) & 3;
+}
 
 // FP16 rows m0 + 4r (r < R, below Mt) of codes k0 .. k0+255, 16 bytes per lane.
 template <int R>
@@ -606,7 +618,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     const int Mt = min(T, M - mt * T);
     if constexpr (FUSEDQ) {
       grid_wait_dependencies();                   // the activations may come from the previous kernel
-      load_act_rows<R>(xv, xt, Mt, K, q, kb0 * kKBlock, lane);
+      load_act_rows<R>(xv, xt, Mt, K, fq_row0(q, 0, Mt), kb0 * kKBlock, lane);
     }
     for (int i = 0; i < nst; ++i) {
       if constexpr (FUSEDQ) {
@@ -620,7 +632,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         uint4 cur[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) cur[r] = xv[r];
-        quantize_act_rows<T, R, kQaRowsTogether>(cur, Mt, q, gs_log2, args.qmax,
+        quantize_act_rows<T, R, kQaRowsTogether>(cur, Mt, fq_row0(q, i, Mt), gs_log2, args.qmax,
                                                  xs_ring + st.idx * Cfg::kXsBytes,
                                                  qa_ring + qp.idx * FusedQLayout<T>::kSlotHalves,
                                                  lane);
@@ -666,7 +678,8 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       if (lane == 0) mbar_arrive(&ctrl->a_full[as.idx]);
       // fused quantization: the next stage's rows, requested once this
       // stage's weights are out of the registers
-      if (FUSEDQ && i + 1 < nst) load_act_rows<R>(xv, xt, Mt, K, q, (kb0 + 2 * i + 2) * kKBlock, lane);
+      if (FUSEDQ && i + 1 < nst)
+        load_act_rows<R>(xv, xt, Mt, K, fq_row0(q, i + 1, Mt), (kb0 + 2 * i + 2) * kKBlock, lane);
       st.next();
       as.next();
     }

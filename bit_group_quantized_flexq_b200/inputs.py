@@ -13,8 +13,8 @@ of the same shapes are used):
   channels (the same for every row) multiplied by ``outlier_scale`` before
   the FP16 cast: 1% x20, or 0.5% x50 for the 70B shapes.
 
-All draws use torch's CPU generator so that every consumer sees identical
-bits for a given seed.
+Draws use torch's CPU generator so that every consumer sees identical bits
+for a given seed (weights may also be drawn on a CUDA device, see weights).
 """
 
 import math
@@ -36,6 +36,15 @@ LLAMA2_13B_M = [1, 64, 4096]
 # (name, N, K, activation bits)
 LLAMA2_70B_LAYERS = [("q_o", 8192, 8192, 6), ("gate_up", 28672, 8192, 6),
                      ("down", 8192, 28672, 8)]
+# One LLaMA-2-70B transformer block, layer by layer: (name, N, K, input site).
+# k and v are 1024 wide (8 key/value heads of 128 under grouped-query
+# attention); layers with the same site read the same activations.
+LLAMA2_70B_BLOCK = [
+    ("q", 8192, 8192, "attn_in"), ("k", 1024, 8192, "attn_in"), ("v", 1024, 8192, "attn_in"),
+    ("o", 8192, 8192, "attn_out"),
+    ("gate", 28672, 8192, "mlp_in"), ("up", 28672, 8192, "mlp_in"),
+    ("down", 8192, 28672, "mlp_act"),
+]
 LLAMA2_70B_M = [1, 16, 512, 8192]
 
 SWEEP_NK = 8192
@@ -49,8 +58,18 @@ def _gen(seed):
     return g
 
 
-def weights(N, K, std=0.02, seed=0):
-    """FP16 [N, K] drawn from N(0, std)."""
+def weights(N, K, std=0.02, seed=0, device="cpu"):
+    """FP16 [N, K] drawn from N(0, std).  With a CUDA device the draw uses that
+    device's generator (fast for the largest layers; its bits differ from the
+    CPU draw of the same seed, so use it only where no oracle comparison
+    follows)."""
+    dev = torch.device(device)
+    if dev.type == "cuda":
+        g = torch.Generator(device=dev)
+        g.manual_seed(int(seed))
+        w = torch.randn(N, K, generator=g, dtype=torch.float32, device=dev)
+        w.mul_(std)
+        return w.to(torch.float16)
     w = torch.randn(N, K, generator=_gen(seed), dtype=torch.float32) * std
     return w.to(torch.float16)
 

@@ -180,10 +180,11 @@ size_t flexq_linear_workspace_bytes(int M, int N, int K, int group_size);
 
 /*
  * flexq_linear_launches -- kernel launches of one linear call for a shape:
- * 1 where the activations are quantized inside the GEMM (batches of at most
- * 2 tokens on 16-token tiles, the sizes where that is not slower than a
- * separate quantizer), 2 otherwise (quantizer, GEMM).  0 for unsupported
- * shapes and M <= 0.  Pure host computation.
+ * 1 where the activations are quantized inside the GEMM, 2 otherwise
+ * (quantizer, GEMM).  The GEMM quantizes on 16-token tiles whose CTAs each
+ * stream few stages of 256 codes of K: at most 4 for up to 4 tokens, at most
+ * 2 for up to 8 tokens (where it is faster than a separate quantizer).
+ * 0 for unsupported shapes and M <= 0.  Pure host computation.
  */
 int flexq_linear_launches(int M, int N, int K, int group_size);
 
@@ -207,9 +208,10 @@ int flexq_linear_launches(int M, int N, int K, int group_size);
  *                    quantization runs inside the GEMM, NULL with 0 bytes
  *                    runs without a K split, as for the GEMM; elsewhere the
  *                    workspace is required (FLEXQ_ERR_INVALID_ARG).
- * Batches of at most 2 tokens quantize the activations inside the GEMM
- * kernel (one launch, no quantized copy in device memory); larger ones launch
- * the activation quantizer into the workspace and then the GEMM.  Both routes
+ * Small batches on short K ranges (flexq_linear_launches) quantize the
+ * activations inside the GEMM kernel (one launch, no quantized copy in device
+ * memory); the others launch the activation quantizer into the workspace and
+ * then the GEMM.  Both routes
  * compute the same codes and scales as flexq_quantize_act, and the result is
  * bit-identical to flexq_quantize_act followed by flexq_gemm_w6a6/w6a8 under
  * the same plan.

@@ -1,0 +1,81 @@
+"""The mixed W6A6 / W6A8 layer stack on the GPU: every layer's output is
+bit-identical to flexq.linear on that layer alone (the stack only shares the
+quantization of a site between layers of the same bit width), and within the
+GEMM tolerance of the oracle's linear layer."""
+
+import pytest
+import torch
+
+from bit_group_quantized_flexq_b200 import flexq, inputs, stack
+from oracle import flexq_oracle as orc
+from tests.gpu_util import assert_within, np16
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-3
+
+# the 70B block with every width divided by 8 (same structure, quick oracle)
+SMALL = [(n, N // 8, K // 8, site) for (n, N, K, site) in inputs.LLAMA2_70B_BLOCK]
+MIXED = {"group_size": 128,
+         "act_bits": {"q": 6, "k": 8, "v": 6, "o": 8, "gate": 6, "up": 6, "down": 8}}
+
+
+def _acts(layers, M, seed):
+    sites = {}
+    for name, N, K, site in layers:
+        sites.setdefault(site, K)
+    return {site: inputs.activations(M, K, outlier_frac=0.005, outlier_scale=50.0,
+                                     seed=inputs.layer_seed("stack-x", seed, site))
+            for site, K in sites.items()}
+
+
+@pytest.mark.parametrize("M", [1, 5, 40])
+def test_small_block_matches_single_layers_and_the_oracle(M):
+    w = {name: inputs.weights(N, K, std=0.015, seed=inputs.layer_seed("stack-w", name))
+         for name, N, K, _ in SMALL}
+    st = stack.LayerStack(SMALL, MIXED, weights=w)
+    acts = _acts(SMALL, M, seed=M)
+    dacts = {k: v.cuda() for k, v in acts.items()}
+    out = st.forward(dacts)
+    for name, N, K, site in SMALL:
+        wp, ws = st.packed[name]
+        bits = MIXED["act_bits"][name]
+        alone = flexq.linear(dacts[site], wp, ws, N, 128, bits)
+        assert torch.equal(out[name], alone), name
+        ref = orc.linear_layer(acts[site].numpy(), w[name].numpy(), 128, bits)
+        assert_within(np16(out[name]), ref["y64"], TOL)
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_70b_block_matches_single_layers(M):
+    st = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED)
+    acts = {k: v.cuda() for k, v in _acts(inputs.LLAMA2_70B_BLOCK, M, seed=70).items()}
+    out = st.forward(acts)
+    for name, N, K, site in inputs.LLAMA2_70B_BLOCK:
+        wp, ws = st.packed[name]
+        alone = flexq.linear(acts[site], wp, ws, N, 128, st.bits[name])
+        assert torch.equal(out[name], alone), name
+    assert flexq.device_status()[0] == flexq.FLEXQ_OK
+
+
+def test_launch_count_shares_site_quantization():
+    st = stack.LayerStack(SMALL, MIXED)
+    assert st.launches(1) == 7                       # quantization inside each GEMM
+    # M = 40: attn_in has 6-bit q, v and 8-bit k (2 quantizations + 3 GEMMs),
+    # attn_out 2, mlp_in 1 + 2, mlp_act 2
+    assert st.launches(40) == 5 + 2 + 3 + 2
+    # the 70B block at M = 1: q (8 stages per CTA) quantizes attn_in for k and
+    # v too; o, gate and down quantize first; up reuses gate's codes
+    big = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED)
+    assert big.launches(1) == 2 + 1 + 1 + 2 + 2 + 1 + 2
+
+
+def test_forward_rejects_mismatched_sites():
+    st = stack.LayerStack(SMALL, MIXED)
+    acts = {k: v.cuda() for k, v in _acts(SMALL, 4, seed=1).items()}
+    acts["mlp_act"] = acts["mlp_act"][:3]
+    with pytest.raises(ValueError, match="same number of tokens"):
+        st.forward(acts)
+    acts["mlp_act"] = torch.zeros(4, 100, dtype=torch.float16, device="cuda")
+    with pytest.raises(ValueError, match="must be"):
+        st.forward(acts)
