@@ -600,10 +600,28 @@ def stack_diagnostics(device, hbm_gbs, int8_peak_tops, ms=(1, 16, 512, 8192)):
     block (q, k, v, o, gate, up, down; 8-bit activations for down), seeded
     synthetic weights drawn on the device: per M, the device time of one
     block forward from FP16 activations (CUDA graph of a few forwards), with
-    the HBM roofline for M <= 16 and the int8 roofline above."""
+    the HBM roofline for M <= 16 and the int8 roofline above; once with
+    every layer its own GEMM, once with q/k/v and gate/up merged
+    (fuse_sites)."""
     import torch
-    from bit_group_quantized_flexq_b200 import flexq, inputs, stack
-    st = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED, device=device)
+    from bit_group_quantized_flexq_b200 import inputs, stack
+    res = {}
+    for fuse in (False, True):
+        st = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED, device=device,
+                              fuse_sites=fuse)
+        res["fused_sites" if fuse else "layers"] = _stack_rows(st, device, hbm_gbs,
+                                                               int8_peak_tops, ms)
+        bits, gs, packed = st.bits, st.gs, st.packed_bytes()
+        del st
+        torch.cuda.empty_cache()
+    return {"block": "LLaMA-2-70B (q, k, v, o, gate, up, down)",
+            "act_bits": bits, "group_size": gs, "packed_MB": round(packed / 1e6, 1),
+            "by_m": res["layers"], "by_m_fused_sites": res["fused_sites"]}
+
+
+def _stack_rows(st, device, hbm_gbs, int8_peak_tops, ms):
+    import torch
+    from bit_group_quantized_flexq_b200 import inputs
     stream = torch.cuda.Stream(device)
     rows = []
     for M in ms:
@@ -624,9 +642,7 @@ def stack_diagnostics(device, hbm_gbs, int8_peak_tops, ms=(1, 16, 512, 8192)):
                      "frac": round(gbs / hbm_gbs if bound == "hbm" else tops / int8_peak_tops, 4),
                      "launches": st.launches(M)})
         del acts, out
-    return {"block": "LLaMA-2-70B (q, k, v, o, gate, up, down)",
-            "act_bits": st.bits, "group_size": st.gs,
-            "packed_MB": round(st.packed_bytes() / 1e6, 1), "by_m": rows}
+    return rows
 
 
 def int8_library_context(W, device, M, reps=20):

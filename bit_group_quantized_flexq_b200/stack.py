@@ -14,6 +14,15 @@ GEMM (flexq.linear_launches == 1), flexq.linear; otherwise the site is
 quantized once (flexq.quantize_act) for this and later layers.  Every output
 is bit-identical to flexq.linear on that layer alone.
 
+With fuse_sites=True the layers of one site and width are also merged into
+one GEMM (the fused q/k/v and gate/up projections of inference engines):
+their FP16 weights are stacked along N and quantized as one matrix (the
+quantization is per row, so every layer keeps its codes and scales), and
+each layer's output is its column slice of the merged output.  One launch
+then carries several layers' set-up and split-K tail; each output equals
+flexq.linear on the stacked weights, and differs from the layer run alone
+only in the FP32 summation order of a different K split.
+
 Configuration (a dict, or a JSON file holding one):
 
     {"group_size": 128,
@@ -68,29 +77,51 @@ def parse_config(cfg, layers):
 class LayerStack:
     """Packed weights of a stack of linear layers and the per-layer bits.
 
-    layers:  [(name, N, K, site)], e.g. inputs.LLAMA2_70B_BLOCK;
-    config:  see the module docstring;
-    weights: {name: FP16 [N, K] tensor} (any device), or None for seeded
-             synthetic weights drawn on `device` (N(0, std)).
+    layers:     [(name, N, K, site)], e.g. inputs.LLAMA2_70B_BLOCK;
+    config:     see the module docstring;
+    weights:    {name: FP16 [N, K] tensor} (any device), or None for seeded
+                synthetic weights drawn on `device` (N(0, std));
+    fuse_sites: merge the layers of one site and width into one GEMM.
     """
 
-    def __init__(self, layers, config, device="cuda", weights=None, std=0.015, seed=0):
+    def __init__(self, layers, config, device="cuda", weights=None, std=0.015, seed=0,
+                 fuse_sites=False):
         self.layers = list(layers)
         self.gs, self.bits = parse_config(config, self.layers)
         self.device = torch.device(device)
+        self.fuse_sites = fuse_sites
         self.site_k = {}
         for name, N, K, site in self.layers:
             if self.site_k.setdefault(site, K) != K:
                 raise ValueError(f"site {site!r} read with K = {self.site_k[site]} and {K}")
-        self.packed = {}
-        for name, N, K, _ in self.layers:
+
+        def weight(name, N, K):
             if weights is not None:
-                w = weights[name].to(self.device)
+                return weights[name].to(self.device)
+            return inputs.weights(N, K, std=std, seed=inputs.layer_seed("stack", seed, name),
+                                  device=self.device)
+
+        # units of work in layer order: one layer, or (fuse_sites) all layers
+        # of a (site, bits) pair, stacked along N at the first one's place
+        self.units = []                    # (key, site, bits, K, [(name, N, offset)], N_total)
+        by_key = {}
+        for name, N, K, site in self.layers:
+            key = (site, self.bits[name]) if fuse_sites else name
+            if key not in by_key:
+                by_key[key] = len(self.units)
+                self.units.append([key, site, self.bits[name], K, [], 0])
+            u = self.units[by_key[key]]
+            u[4].append((name, N, u[5]))
+            u[5] += N
+        self.packed = {}                   # unit key -> (packed weights, scales)
+        for key, site, bits, K, members, n_total in self.units:
+            if len(members) == 1:
+                w = weight(members[0][0], members[0][1], K)
             else:
-                w = inputs.weights(N, K, std=std, seed=inputs.layer_seed("stack", seed, name),
-                                   device=self.device)
-            self.packed[name] = flexq.quantize_weight(w, self.gs)
+                w = torch.cat([weight(name, N, K) for name, N, _ in members], dim=0)
+            self.packed[key] = flexq.quantize_weight(w, self.gs)
             del w
+        self._ybuf = {}
 
     def sites(self):
         """{site: K}: the activations the stack reads."""
@@ -99,21 +130,32 @@ class LayerStack:
     def packed_bytes(self):
         return sum(wp.numel() + ws.numel() * 2 for wp, ws in self.packed.values())
 
+    def layer_weights(self, name):
+        """(packed weights, scales, N) that produce layer `name`: its own, or
+        its merged unit's (fuse_sites; the layer is a column slice of it)."""
+        for key, site, bits, K, members, n_total in self.units:
+            if any(m[0] == name for m in members):
+                wp, ws = self.packed[key]
+                return wp, ws, n_total
+        raise KeyError(name)
+
     def launches(self, M):
         """Kernel launches of one forward at batch M."""
         n, quantized = 0, set()
-        for name, N, K, site in self.layers:
-            key = (site, self.bits[name])
-            if key in quantized or flexq.linear_launches(M, N, K, self.gs) == 1:
+        for key, site, bits, K, members, n_total in self.units:
+            q = (site, bits)
+            if q in quantized or flexq.linear_launches(M, n_total, K, self.gs) == 1:
                 n += 1
             else:
                 n += 2
-                quantized.add(key)
+                quantized.add(q)
         return n
 
     def forward(self, acts, out=None):
         """acts: {site: FP16 [M, K]} on the stack's device.  Returns
-        {layer name: FP16 [M, N]} (written into `out` when given)."""
+        {layer name: FP16 [M, N]}: written into `out` for layers run alone
+        when given; merged layers (fuse_sites) are column views of a buffer
+        the stack keeps per batch size."""
         M = None
         for site, K in self.site_k.items():
             x = acts[site]
@@ -125,16 +167,26 @@ class LayerStack:
                 raise ValueError("every site must hold the same number of tokens")
         out = {} if out is None else out
         codes = {}
-        for name, N, K, site in self.layers:
-            wp, ws = self.packed[name]
-            bits = self.bits[name]
-            y = out.get(name)
-            key = (site, bits)
-            if key not in codes and flexq.linear_launches(M, N, K, self.gs) == 1:
-                out[name] = flexq.linear(acts[site], wp, ws, N, self.gs, bits, out=y)
-                continue
-            if key not in codes:
-                codes[key] = flexq.quantize_act(acts[site], self.gs, bits)
-            xq, xs = codes[key]
-            out[name] = flexq.gemm(xq, xs, wp, ws, N, self.gs, bits, out=y)
+        for key, site, bits, K, members, n_total in self.units:
+            wp, ws = self.packed[key]
+            if len(members) == 1:
+                y = out.get(members[0][0])
+            else:                          # merged unit: one buffer per batch size
+                y = self._ybuf.get((key, M))
+                if y is None:
+                    y = torch.empty(M, n_total, dtype=torch.float16, device=self.device)
+                    self._ybuf[(key, M)] = y
+            q = (site, bits)
+            if q not in codes and flexq.linear_launches(M, n_total, K, self.gs) == 1:
+                y = flexq.linear(acts[site], wp, ws, n_total, self.gs, bits, out=y)
+            else:
+                if q not in codes:
+                    codes[q] = flexq.quantize_act(acts[site], self.gs, bits)
+                xq, xs = codes[q]
+                y = flexq.gemm(xq, xs, wp, ws, n_total, self.gs, bits, out=y)
+            if len(members) == 1:
+                out[members[0][0]] = y
+            else:
+                for name, N, off in members:
+                    out[name] = y[:, off:off + N]
         return out

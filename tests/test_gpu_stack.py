@@ -38,7 +38,7 @@ def test_small_block_matches_single_layers_and_the_oracle(M):
     dacts = {k: v.cuda() for k, v in acts.items()}
     out = st.forward(dacts)
     for name, N, K, site in SMALL:
-        wp, ws = st.packed[name]
+        wp, ws, _ = st.layer_weights(name)
         bits = MIXED["act_bits"][name]
         alone = flexq.linear(dacts[site], wp, ws, N, 128, bits)
         assert torch.equal(out[name], alone), name
@@ -52,7 +52,7 @@ def test_70b_block_matches_single_layers(M):
     acts = {k: v.cuda() for k, v in _acts(inputs.LLAMA2_70B_BLOCK, M, seed=70).items()}
     out = st.forward(acts)
     for name, N, K, site in inputs.LLAMA2_70B_BLOCK:
-        wp, ws = st.packed[name]
+        wp, ws, _ = st.layer_weights(name)
         alone = flexq.linear(acts[site], wp, ws, N, 128, st.bits[name])
         assert torch.equal(out[name], alone), name
     assert flexq.device_status()[0] == flexq.FLEXQ_OK
@@ -79,3 +79,35 @@ def test_forward_rejects_mismatched_sites():
     acts["mlp_act"] = torch.zeros(4, 100, dtype=torch.float16, device="cuda")
     with pytest.raises(ValueError, match="must be"):
         st.forward(acts)
+
+
+@pytest.mark.parametrize("M", [1, 4, 40])
+def test_fused_sites_match_the_stacked_layer_and_the_oracle(M):
+    w = {name: inputs.weights(N, K, std=0.015, seed=inputs.layer_seed("stack-w", name))
+         for name, N, K, _ in SMALL}
+    cfg = {"group_size": 128,
+           "act_bits": {"q": 6, "k": 6, "v": 8, "o": 8, "gate": 6, "up": 6, "down": 8}}
+    st = stack.LayerStack(SMALL, cfg, weights=w, fuse_sites=True)
+    # q and k merge (v has other bits); gate and up merge
+    assert [len(u[4]) for u in st.units] == [2, 1, 1, 2, 1]
+    acts = _acts(SMALL, M, seed=M + 7)
+    dacts = {k: v.cuda() for k, v in acts.items()}
+    out = st.forward(dacts)
+    for name, N, K, site in SMALL:
+        bits = cfg["act_bits"][name]
+        wp, ws, n_total = st.layer_weights(name)
+        merged = flexq.linear(dacts[site], wp, ws, n_total, 128, bits)
+        off = [m for u in st.units for m in u[4] if m[0] == name][0][2]
+        assert torch.equal(out[name], merged[:, off:off + N]), name
+        ref = orc.linear_layer(acts[site].numpy(), w[name].numpy(), 128, bits)
+        assert_within(np16(out[name]), ref["y64"], TOL)
+
+
+def test_fused_70b_block_launches():
+    st = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED, fuse_sites=True)
+    assert [len(u[4]) for u in st.units] == [3, 1, 2, 1]      # qkv, o, gate+up, down
+    assert st.launches(16) == 4 * 2
+    acts = {k: v.cuda() for k, v in _acts(inputs.LLAMA2_70B_BLOCK, 16, seed=71).items()}
+    out = st.forward(acts)
+    assert out["k"].shape == (16, 1024) and out["up"].shape == (16, 28672)
+    assert flexq.device_status()[0] == flexq.FLEXQ_OK
