@@ -14,7 +14,7 @@ Output: one JSON line (rank 0).  `value` is whole-job TOPS (2*M*N*K summed over
 the step, divided by the device time), measured over CUDA-graph replays of the
 step with inputs resident in HBM; `e2e` is the same metric through the public
 Python API with host buffers (pinned H2D copy of every layer input, D2H copy of
-every output) inside the timed region.
+every output) inside the timed region, copies and layer calls on three streams.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl flexq|reference]
 
@@ -683,38 +683,71 @@ def int8_library_context(W, device, M, reps=20):
 def run_e2e(W, args, device, world):
     """The same metric through the public API with host buffers: every step
     copies each layer's FP16 input from pinned host memory and each output
-    back to pinned host memory."""
+    back to pinned host memory.  Copies in, layer calls and copies out run
+    on three streams joined by events (each layer waits for its input, each
+    copy out for its layer; a buffer is refilled only after its last reader
+    of the previous step), so the two copy directions and the kernels
+    overlap as the hardware's copy engines allow."""
     import torch
     from bit_group_quantized_flexq_b200 import flexq
-    hx = {k: v.cpu().pin_memory() for k, v in W.x.items()}
+    keys = [(M, layer) for M in W.ms for layer in W.w]
+    hx = {(M, l[0]): W.x[(M, l[2])].cpu().pin_memory() for M, l in keys}
     hy = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in W.y.items()}
-    dx = {k: torch.empty_like(v) for k, v in W.x.items()}
-    h2d = sum(W.x[(M, K)].numel() * 2 for M in W.ms for (_, _, K, _, _) in W.w)
+    dx = {(M, l[0]): torch.empty_like(W.x[(M, l[2])]) for M, l in keys}
+    h2d = sum(v.numel() * 2 for v in hx.values())
     d2h = sum(v.numel() * 2 for v in W.y.values())
+    s_in, s_c, s_out = (torch.cuda.Stream(device) for _ in range(3))
+    ev = lambda: torch.cuda.Event()
+    done_in = {k: ev() for k in hx}
+    done_c = {k: ev() for k in hx}
+    done_out = {k: ev() for k in hx}
+    started = [False]
 
     def step():
-        for M in W.ms:
-            for (name, N, K, wp, ws) in W.w:
-                dx[(M, K)].copy_(hx[(M, K)], non_blocking=True)
-                flexq.linear(dx[(M, K)], wp, ws, N, GS, ACT_BITS, out=W.y[(M, name)])
-                hy[(M, name)].copy_(W.y[(M, name)], non_blocking=True)
+        for M, (name, N, K, wp, ws) in keys:
+            k = (M, name)
+            if started[0]:
+                s_in.wait_event(done_c[k])        # the previous step's layer has read dx
+            with torch.cuda.stream(s_in):
+                dx[k].copy_(hx[k], non_blocking=True)
+                done_in[k].record(s_in)
+            s_c.wait_event(done_in[k])
+            if started[0]:
+                s_c.wait_event(done_out[k])       # the previous step's copy out has read y
+            with torch.cuda.stream(s_c):
+                flexq.linear(dx[k], wp, ws, N, GS, ACT_BITS, out=W.y[k])
+                done_c[k].record(s_c)
+            s_out.wait_event(done_c[k])
+            with torch.cuda.stream(s_out):
+                hy[k].copy_(W.y[k], non_blocking=True)
+                done_out[k].record(s_out)
+        started[0] = True
 
-    for _ in range(args.warmup):
-        step()
+    main = torch.cuda.current_stream(device)
+
+    def run(n):
+        for stream in (s_in, s_c, s_out):
+            stream.wait_stream(main)
+        for _ in range(n):
+            step()
+        for stream in (s_in, s_c, s_out):
+            main.wait_stream(stream)
+
+    run(args.warmup)
     torch.cuda.synchronize(device)
     barrier(device)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(args.steps):
-        step()
-    t1.record()
+    t0.record(main)
+    run(args.steps)
+    t1.record(main)
     torch.cuda.synchronize(device)
     t_max = max_over_ranks(t0.elapsed_time(t1) / 1e3, device)
     ops = step_ops(W.ms, [(n, N, K) for (n, N, K, _, _) in W.w])
     return {"value": round(aggregate(ops * args.steps, world, t_max) / 1e12, 3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "ms_per_step": round(t_max * 1e3 / args.steps, 4)}
+            "ms_per_step": round(t_max * 1e3 / args.steps, 4),
+            "streams": "copies in, layer calls and copies out on three streams"}
 
 
 # ------------------------------------------------------- CPU oracle arm ----
