@@ -836,13 +836,19 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         part[(static_cast<size_t>(ks) * T + col0 + j) * kTileRows + row] =
             (j & 1) ? acc[j / 2].y : acc[j / 2].x;
     }
-    __threadfence();
     __syncthreads();
     FLEXQ_CTA_TIME(6);
     if (threadIdx.x == 0) {
+      // the barrier orders the CTA's partial stores before this thread's
+      // fence, which releases them with the count; the last CTA's fence
+      // acquires the other CTAs' partials before the barrier below
+      __threadfence();
       const unsigned old = atomicAdd(&args.ws_cnt[st_idx], 1u);
       const bool last = old == static_cast<unsigned>(S - 1);
-      if (last) args.ws_cnt[st_idx] = 0u;
+      if (last) {
+        args.ws_cnt[st_idx] = 0u;
+        __threadfence();
+      }
       ctrl->is_last = last ? 1u : 0u;
     }
     __syncthreads();
@@ -850,7 +856,6 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       FLEXQ_CTA_TIME(3);
       return;
     }
-    __threadfence();
     if (is_epi) {
       float2 sum[Cfg::kCols / 2];
 #pragma unroll
