@@ -486,6 +486,16 @@ def run_flexq(args, rank, world):
     runners.clear()
 
 
+def roofline(ops, nbytes, us, hbm_gbs, int8_peak_tops):
+    """(bound, fraction) of a launch against the attainable rate
+    min(int8 peak, HBM bandwidth x ops per algorithmic byte)."""
+    intensity = ops / nbytes
+    mem_tops = hbm_gbs * 1e9 * intensity / 1e12
+    bound = "hbm" if mem_tops < int8_peak_tops else "tensor"
+    achieved = ops / (us * 1e-6) / 1e12
+    return bound, achieved / min(mem_tops, int8_peak_tops)
+
+
 def linear_bytes(M, N, K, gs=GS):
     """Algorithmic HBM bytes of one whole linear layer from FP16 activations:
     packed weights, weight scales, FP16 activations read once, FP16 output."""
@@ -515,7 +525,8 @@ def _graph_time_us(body, device, stream, reps):
 
 
 def gemm_diagnostics(W, device, hbm_gbs, int8_peak_tops, reps=10):
-    """Per-M times and roofline fractions (HBM bound for M <= 16, tensor bound
+    """Per-M times and fractions of the attainable roofline (min(int8 peak,
+    HBM x intensity): HBM-bound at decode sizes, tensor-bound at M = 256 and
     above) of the seven layers, each timed from a CUDA graph that holds `reps`
     rounds of them back to back (the other layers' weights stream in between,
     so each launch reads its weights cold); events bracket the graph replay,
@@ -543,16 +554,17 @@ def gemm_diagnostics(W, device, hbm_gbs, int8_peak_tops, reps=10):
         t_us = _graph_time_us(gemm_body, device, stream, reps)
         l_us = _graph_time_us(linear_body, device, stream, reps)
         flops = sum(2.0 * M * N * K for (_, N, K, _, _) in W.w)
-        bound = "hbm" if M <= 16 else "tensor"
-        row = {"M": M, "bound": bound}
+        row = {"M": M}
         for key, us, nbytes in (("gemm", t_us, sum(gemm_bytes(M, N, K) for (_, N, K, _, _) in W.w)),
                                 ("linear", l_us, sum(linear_bytes(M, N, K) for (_, N, K, _, _) in W.w))):
             gbs = nbytes / (us * 1e-6) / 1e9
             tops = flops / (us * 1e-6) / 1e12
+            bound, frac = roofline(flops, nbytes, us, hbm_gbs, int8_peak_tops)
+            row["bound"] = bound
             row[f"{key}_us"] = round(us, 2)
             row[f"{key}_GB/s"] = round(gbs, 1)
             row[f"{key}_TOPS"] = round(tops, 2)
-            row[f"{key}_frac"] = round(gbs / hbm_gbs if bound == "hbm" else tops / int8_peak_tops, 4)
+            row[f"{key}_frac"] = round(frac, 4)
         row["plan"] = [list(flexq.plan(M, N, K, GS)) for (_, N, K, _, _) in W.w]
         out.append(row)
     return out
@@ -600,7 +612,7 @@ def stack_diagnostics(device, hbm_gbs, int8_peak_tops, ms=(1, 16, 512, 8192)):
     block (q, k, v, o, gate, up, down; 8-bit activations for down), seeded
     synthetic weights drawn on the device: per M, the device time of one
     block forward from FP16 activations (CUDA graph of a few forwards), with
-    the HBM roofline for M <= 16 and the int8 roofline above; once with
+    the attainable roofline min(int8 peak, HBM x intensity); once with
     every layer its own GEMM, once with q/k/v and gate/up merged
     (fuse_sites)."""
     import torch
@@ -634,15 +646,79 @@ def _stack_rows(st, device, hbm_gbs, int8_peak_tops, ms):
         us = _graph_time_us(lambda: st.forward(acts, out), device, stream, reps)
         flops = sum(2.0 * M * N * K for _, N, K, _ in st.layers)
         nbytes = sum(linear_bytes(M, N, K, st.gs) for _, N, K, _ in st.layers)
-        bound = "hbm" if M <= 16 else "tensor"
         gbs = nbytes / (us * 1e-6) / 1e9
         tops = flops / (us * 1e-6) / 1e12
+        bound, frac = roofline(flops, nbytes, us, hbm_gbs, int8_peak_tops)
         rows.append({"M": M, "us": round(us, 2), "TOPS": round(tops, 2), "GB/s": round(gbs, 1),
-                     "bound": bound,
-                     "frac": round(gbs / hbm_gbs if bound == "hbm" else tops / int8_peak_tops, 4),
-                     "launches": st.launches(M)})
+                     "bound": bound, "frac": round(frac, 4), "launches": st.launches(M)})
         del acts, out
     return rows
+
+
+def run_sweep(device, hbm_gbs, int8_peak_tops):
+    """The other measured configurations, one JSON line (`--sweep`; not part
+    of the default run): the LLaMA-2-13B W6A8 layers at M in {1, 64, 4096}
+    and the N = K = 8192 sweep over group size {32, 64, 128, 256}, W6A6 and
+    W6A8, M in {1, 8, 32, 128, 1024, 4096, 16384}.  Per case the GEMM alone
+    (codes given) and the whole layer from FP16 activations (flexq.linear),
+    device time per call from a CUDA graph that rotates over enough copies
+    of the packed weights to exceed L2, against the attainable rate
+    min(int8 peak, HBM bandwidth x arithmetic intensity)."""
+    import torch
+    from bit_group_quantized_flexq_b200 import flexq, inputs
+    stream = torch.cuda.Stream(device)
+
+    def case(M, N, K, gs, bits, wp0, ws0, copies):
+        x = inputs.activations(M, K, outlier_frac=0.01, outlier_scale=20.0,
+                               seed=inputs.layer_seed("sweep-x", M, K)).to(device)
+        xq, xs = flexq.quantize_act(x, gs, bits)
+        y = torch.empty(M, N, dtype=torch.float16, device=device)
+        reps = 1 if M >= 4096 else 3
+
+        def gemm():
+            for wp, ws in copies:
+                flexq.gemm(xq, xs, wp, ws, N, gs, bits, out=y)
+
+        def lin():
+            for wp, ws in copies:
+                flexq.linear(x, wp, ws, N, gs, bits, out=y)
+        row = {"M": M, "N": N, "K": K, "gs": gs, "act_bits": bits,
+               "plan": list(flexq.plan(M, N, K, gs)),
+               "linear_launches": flexq.linear_launches(M, N, K, gs)}
+        for key, body, nbytes in (("gemm", gemm, gemm_bytes(M, N, K, gs)),
+                                  ("linear", lin, linear_bytes(M, N, K, gs))):
+            us = _graph_time_us(body, device, stream, reps) / len(copies)
+            tops = 2.0 * M * N * K / (us * 1e-6) / 1e12
+            bound, frac = roofline(2.0 * M * N * K, nbytes, us, hbm_gbs, int8_peak_tops)
+            row[f"{key}_us"] = round(us, 2)
+            row[f"{key}_TOPS"] = round(tops, 2)
+            row[f"{key}_frac"] = round(frac, 4)
+            row["bound"] = bound
+        del x, xq, xs, y
+        return row
+
+    def weights(N, K, gs, std):
+        w = inputs.weights(N, K, std=std, seed=inputs.layer_seed("sweep-w", N, K), device=device)
+        wp, ws = flexq.quantize_weight(w, gs)
+        del w
+        n = max(2, int((400 << 20) // wp.numel()) + 1)
+        return wp, ws, [(wp, ws)] + [(wp.clone(), ws.clone()) for _ in range(n - 1)]
+
+    out = {"13b_w6a8": [], "sweep_8192": []}
+    for N, K in [(5120, 5120), (13824, 5120), (5120, 13824)]:
+        wp, ws, copies = weights(N, K, 128, 0.02)
+        for M in (1, 64, 4096):
+            out["13b_w6a8"].append(case(M, N, K, 128, 8, wp, ws, copies))
+        del copies
+        torch.cuda.empty_cache()
+    for gs in (32, 64, 128, 256):
+        wp, ws, copies = weights(8192, 8192, gs, 0.02)
+        for bits in (6, 8):
+            for M in (1, 8, 32, 128, 1024, 4096, 16384):
+                out["sweep_8192"].append(case(M, 8192, 8192, gs, bits, wp, ws, copies))
+        del copies
+        torch.cuda.empty_cache()
+    return out
 
 
 def int8_library_context(W, device, M, reps=20):
@@ -844,6 +920,9 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     p.add_argument("--no-diag", dest="diag", action="store_false")
     p.add_argument("--cpu-budget-s", type=float, default=20.0)
+    p.add_argument("--sweep", action="store_true",
+                   help="measure the 13B W6A8 layers and the N = K = 8192 group-size sweep "
+                        "instead of the step (one JSON line)")
     a = p.parse_args(argv)
     if a.warmup < 3 and a.impl == "flexq" and not (a.ms or a.layers):
         p.error("--warmup must be >= 3")
@@ -856,6 +935,17 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.sweep:
+            import torch
+            _, _, local = dist_env()
+            device = torch.device("cuda", local)
+            torch.cuda.set_device(device)
+            peaks, src = measured_peaks()
+            res = run_sweep(device, peaks["hbm_gbs"], peaks["bf16_tflops"] * INT8_OVER_BF16)
+            if rank == 0:
+                print(json.dumps({"sweep": res, "peaks": src,
+                                  "int8_peak_tops": peaks["bf16_tflops"] * INT8_OVER_BF16,
+                                  "hbm_gbs": peaks["hbm_gbs"]}), flush=True)
         else:
             run_flexq(args, rank, world)
     finally:

@@ -168,6 +168,12 @@ Plan make_plan(int M, int N, int K, int gs, int sms, bool partials) {
   Plan p;
   const int units = K / 256;                          // K stages of the kernel
   p.T = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  // 33..64 tokens: two 32-token tiles (each weight tile read twice, the
+  // second time mostly from L2) beat one 64-token tile whenever both fit in
+  // one wave of CTA slots (M = 64: 5120^2 14.9 us against 21.9, 5120x13824
+  // 28.0 against 38.0); with more weight tiles than that (N = 28672) the
+  // 64-token tile keeps one wave and wins
+  if (p.T == 64 && 2LL * (N / 128) <= static_cast<long long>(sms) * min_blocks_for(32)) p.T = 32;
   const int fT = g_force_tokens.load(), fS = g_force_split.load();
   if (fT == 16 || fT == 32 || fT == 64 || fT == 128) p.T = fT;   // any width: more or fewer token tiles
   const long long tiles = static_cast<long long>(N / 128) * ((M + p.T - 1) / p.T);

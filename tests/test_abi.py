@@ -89,7 +89,7 @@ def test_validation_before_any_launch(L):
 
 def test_plan_is_host_only_and_sane(L):
     # tokens per tile follow M; K splits fill the machine at decode sizes
-    for M, T in [(1, 16), (16, 16), (17, 32), (64, 64), (65, 128), (2048, 128)]:
+    for M, T in [(1, 16), (16, 16), (17, 32), (64, 32), (65, 128), (2048, 128)]:
         t, s, c = flexq.plan(M, 4096, 4096, 128)
         assert t == T
         assert 1 <= s <= 8
@@ -111,6 +111,9 @@ def test_plan_is_host_only_and_sane(L):
         t, s, c = flexq.plan(1, N, K, 128)
         assert c <= 2 * 148
     assert flexq.plan(1, 8192, 8192, 128) == (16, 4, 256)
+    # 33..64 tokens: two 32-token tiles while they fit one wave, else one 64-token tile
+    assert flexq.plan(64, 5120, 5120, 128) == (32, 3, 240)
+    assert flexq.plan(64, 28672, 8192, 128)[0] == 64
     assert flexq.plan(0, 256, 256, 128) == (0, 0, 0)
 
 

@@ -136,6 +136,13 @@ FULL = [
     (2048, 4096, 4096, 128, 6, 0.02, 0.01, 20.0),
     (64, 13824, 5120, 128, 8, 0.02, 0.01, 20.0),
     (1, 8192, 28672, 128, 8, 0.015, 0.005, 50.0),
+    # the LLaMA-2-13B W6A8 layers and the N = K = 8192 group-size sweep
+    (4096, 5120, 13824, 128, 8, 0.02, 0.01, 20.0),
+    (1, 5120, 5120, 128, 8, 0.02, 0.01, 20.0),
+    (8, 8192, 8192, 32, 6, 0.02, 0.01, 20.0),
+    (128, 8192, 8192, 64, 8, 0.02, 0.01, 20.0),
+    (1024, 8192, 8192, 256, 6, 0.02, 0.01, 20.0),
+    (16384, 8192, 8192, 32, 8, 0.02, 0.01, 20.0),
 ]
 
 
