@@ -73,3 +73,16 @@ def test_max_over_ranks_two_gloo_ranks():
 def test_single_process_helpers_are_identities():
     assert bench.max_over_ranks(1.5) == 1.5
     bench.barrier()          # no process group: returns without a collective
+
+
+def test_roofline_picks_the_lower_bound():
+    # 4096^2 at M = 1: ~2 ops per byte, far below the ridge -> HBM-bound
+    nb = bench.gemm_bytes(1, 4096, 4096)
+    bound, frac = bench.roofline(2.0 * 4096 * 4096, nb, 10.0, 6500.0, 3300.0)
+    assert bound == "hbm"
+    assert abs(frac - (nb / 10e-6 / 1e9) / 6500.0) < 1e-9          # = achieved GB/s / peak GB/s
+    # 2048 x 4096 x 4096: hundreds of ops per byte -> tensor-bound
+    ops = 2.0 * 2048 * 4096 * 4096
+    bound, frac = bench.roofline(ops, bench.gemm_bytes(2048, 4096, 4096), 100.0, 6500.0, 3300.0)
+    assert bound == "tensor"
+    assert abs(frac - ops / 100e-6 / 1e12 / 3300.0) < 1e-9
