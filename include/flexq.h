@@ -281,10 +281,13 @@ int flexq_debug_group_partials(int M, int N, int K, int group_size,
  * flexq_gemm_plan -- the launch the GEMM entry points would use for a shape
  * given enough workspace: tokens per tile (16, 32, 64 or 128), K-split factor
  * (CTAs that share an output tile, each over its own range of K) and the
- * number of CTAs.  With fewer output tiles than CTA slots every tile is
- * split; otherwise the whole waves of tiles run unsplit and only the tiles of
- * a partial last wave are split (k_split is then their split, 1 if none).
- * Any output pointer may be NULL.  Pure host computation.
+ * number of CTAs.  Tokens per tile follow M (16 up to 16 tokens, 32 up to 32,
+ * 128 above 64; 33..64 tokens take two 32-token tiles while those fit one
+ * wave of CTA slots, else one 64-token tile).  With fewer output tiles than
+ * CTA slots every tile is split (128-token tiles keep at least 8 stages of
+ * 256 codes per CTA); otherwise the whole waves of tiles run unsplit and only
+ * the tiles of a partial last wave are split (k_split is then their split, 1
+ * if none).  Any output pointer may be NULL.  Pure host computation.
  */
 int flexq_gemm_plan(int M, int N, int K, int group_size, int* tile_tokens,
                     int* k_split, int* ctas);
