@@ -1,20 +1,25 @@
 #!/usr/bin/env python
-"""Benchmark of the W6A6 group-quantized linear layers of a LLaMA-2-7B block.
+"""Benchmark of the W6A6 / W6A8 group-quantized linear layers of LLaMA-2-70B.
 
-Workload (one "step"): for every M in {1, 16, 256, 2048} and every linear layer
-of a LLaMA-2-7B transformer block (q, k, v, o: 4096x4096; gate, up: 11008x4096;
-down: 4096x11008), quantize the FP16 activations to 6-bit group codes (group
-size 128) and run the W6A6 group GEMM against 6-bit packed weights.  Inputs are
-seeded synthetic tensors of those shapes (weights N(0, 0.02); activations
-N(0, 1) with 1% outlier channels x20); every step streams 151 MB of distinct
-packed weights, more than the 126 MB L2, so each GEMM reads its weights from
-HBM.
+Workload (one "step"): for every M in {1, 16, 512, 8192} and every linear layer
+of the LLaMA-2-70B configuration -- q and o (8192x8192, 6-bit activations),
+gate and up (28672x8192, 6-bit activations), down (8192x28672, 8-bit
+activations) -- quantize the layer's FP16 activations to group codes (group
+size 128) and run the group GEMM against 6-bit packed weights.  Inputs are
+seeded synthetic tensors of those shapes (weights N(0, 0.015); activations
+N(0, 1) with 0.5% outlier channels x50, one input per site: attention input,
+attention output, MLP input, MLP activation); every step streams 629 MB of
+distinct packed weights per M, far more than the 126 MB L2, so each GEMM reads
+its weights from HBM.
 
 Output: one JSON line (rank 0).  `value` is whole-job TOPS (2*M*N*K summed over
 the step, divided by the device time), measured over CUDA-graph replays of the
-step with inputs resident in HBM; `e2e` is the same metric through the public
-Python API with host buffers (pinned H2D copy of every layer input, D2H copy of
-every output) inside the timed region, copies and layer calls on three streams.
+step with inputs resident in HBM.  `roofline` covers both halves of the
+metric: the tensor-bound GEMM launches at M >= 512 against the int8 peak, and
+the HBM-bound layers at M <= 16 against the measured copy bandwidth.  `e2e` is
+the same metric through the public Python API with host buffers (pinned H2D
+copy of every layer input, D2H copy of every output) inside the timed region,
+copies and layer calls on three streams.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl flexq|reference]
 
@@ -50,15 +55,25 @@ INT8_OVER_BF16 = 2.0          # nominal dense ratio (4.5 vs 2.25 PFLOP/s)
 
 
 # ------------------------------------------------------------- workload ----
+HEADLINE_LAYERS = ("q", "o", "gate", "up", "down")
+WEIGHT_STD = 0.015
+OUTLIER_FRAC, OUTLIER_SCALE = 0.005, 50.0
+TENSOR_MIN_M = 512            # launches at or above this M are tensor-bound
+DECODE_MAX_M = 16             # launches at or below this M are HBM-bound
+
+
 def workload_shapes(ms=None, layers=None):
-    from bit_group_quantized_flexq_b200 import inputs
-    ms = list(ms) if ms else list(inputs.LLAMA2_7B_M)
-    lay = [l for l in inputs.LLAMA2_7B_LAYERS if not layers or l[0] in layers]
+    """M values and [(name, N, K, act_bits, site)] of the LLaMA-2-70B step."""
+    from bit_group_quantized_flexq_b200 import inputs, stack
+    ms = list(ms) if ms else list(inputs.LLAMA2_70B_M)
+    bits = stack.LLAMA2_70B_MIXED["act_bits"]
+    lay = [(n, N, K, bits[n], site) for (n, N, K, site) in inputs.LLAMA2_70B_BLOCK
+           if n in HEADLINE_LAYERS and (not layers or n in layers)]
     return ms, lay
 
 
 def step_ops(ms, layers):
-    return sum(2.0 * M * N * K for M in ms for (_, N, K) in layers)
+    return sum(2.0 * M * l[1] * l[2] for M in ms for l in layers)
 
 
 def gemm_bytes(M, N, K, gs=GS):
@@ -68,8 +83,8 @@ def gemm_bytes(M, N, K, gs=GS):
 
 
 def workload_name(ms, layers):
-    return ("LLaMA-2-7B block W6A6 linear layers ("
-            + ",".join(f"{n}:{N}x{K}" for n, N, K in layers)
+    return ("LLaMA-2-70B linear layers, W6A6 q/o/gate/up + W6A8 down ("
+            + ",".join(f"{l[0]}:{l[1]}x{l[2]}:A{l[3]}" for l in layers)
             + f"), group 128, M in {{{','.join(map(str, ms))}}}")
 
 
@@ -251,78 +266,83 @@ def profiled_traffic():
 
 # ------------------------------------------------------------ flexq arm ----
 class Layers:
-    """Device-resident workload: packed weights, activations, outputs."""
+    """Device-resident workload: packed weights, per-site activations, their
+    codes and scales, outputs.  Layer tuples: (name, N, K, bits, site, wp, ws)."""
 
     def __init__(self, ms, layers, device):
         import torch
         from bit_group_quantized_flexq_b200 import flexq, inputs
         self.ms, self.layers, self.dev = ms, layers, device
         self.w = []
-        for name, N, K in layers:
-            w16 = inputs.weights(N, K, std=0.02, seed=inputs.layer_seed("7b", name)).to(device)
+        for name, N, K, bits, site in layers:
+            w16 = inputs.weights(N, K, std=WEIGHT_STD, seed=inputs.layer_seed("70b", name),
+                                 device=device)
             wp, ws = flexq.quantize_weight(w16, GS)
             del w16
-            self.w.append((name, N, K, wp, ws))
+            self.w.append((name, N, K, bits, site, wp, ws))
         self.x, self.xq, self.xs, self.y = {}, {}, {}, {}
+        sites = {site: K for (_, _, K, _, site) in layers}
         for M in ms:
-            for K in sorted({K for (_, _, K) in layers}):
-                x = inputs.activations(M, K, outlier_frac=0.01, outlier_scale=20.0,
-                                       seed=inputs.layer_seed("7b-x", M, K))
-                self.x[(M, K)] = x.to(device)
-                self.xq[(M, K)] = torch.empty(M, K, dtype=torch.int8, device=device)
-                self.xs[(M, K)] = torch.empty(K // GS, flexq.act_scales_ld(M),
-                                              dtype=torch.float16, device=device)
-            for (name, N, K) in layers:
+            for site, K in sites.items():
+                x = inputs.activations(M, K, outlier_frac=OUTLIER_FRAC,
+                                       outlier_scale=OUTLIER_SCALE,
+                                       seed=inputs.layer_seed("70b-x", M, site))
+                self.x[(M, site)] = x.to(device)
+            for (name, N, K, bits, site, _, _) in self.w:
+                self.xq[(M, name)] = torch.empty(M, K, dtype=torch.int8, device=device)
+                self.xs[(M, name)] = torch.empty(K // GS, flexq.act_scales_ld(M),
+                                                 dtype=torch.float16, device=device)
                 self.y[(M, name)] = torch.empty(M, N, dtype=torch.float16, device=device)
         torch.cuda.synchronize(device)
 
+    def packed_bytes(self):
+        return sum(l[5].numel() for l in self.w)
+
+    def split_m(self, M):
+        """The tensor-bound M run the quantizer and the GEMM as separate
+        launches, so that events bracket every GEMM launch."""
+        return M >= TENSOR_MIN_M
+
     def launches_per_step(self):
-        """Kernel launches of one step: the dominant M runs the quantizer and
-        the GEMM as separate launches (timed apart); the other M run each
-        layer through flexq.linear (one launch where it quantizes inside the
-        GEMM, two otherwise)."""
         from bit_group_quantized_flexq_b200 import flexq
-        dominant = max(self.ms)
         n = 0
         for M in self.ms:
-            for (_, N, K, _, _) in self.w:
-                n += 2 if M == dominant else flexq.linear_launches(M, N, K, GS)
+            for (_, N, K, _, _, _, _) in self.w:
+                n += 2 if self.split_m(M) else flexq.linear_launches(M, N, K, GS)
         return n
 
     def quant(self, M, layer):
         from bit_group_quantized_flexq_b200 import flexq
-        _, _, K, _, _ = layer
-        flexq.quantize_act(self.x[(M, K)], GS, ACT_BITS, out=(self.xq[(M, K)], self.xs[(M, K)]))
+        name, _, _, bits, site, _, _ = layer
+        flexq.quantize_act(self.x[(M, site)], GS, bits,
+                           out=(self.xq[(M, name)], self.xs[(M, name)]))
 
     def gemm(self, M, layer):
         from bit_group_quantized_flexq_b200 import flexq
-        name, N, K, wp, ws = layer
-        flexq.gemm(self.xq[(M, K)], self.xs[(M, K)], wp, ws, N, GS, ACT_BITS,
+        name, N, K, bits, _, wp, ws = layer
+        flexq.gemm(self.xq[(M, name)], self.xs[(M, name)], wp, ws, N, GS, bits,
                    out=self.y[(M, name)])
 
     def linear(self, M, layer):
         from bit_group_quantized_flexq_b200 import flexq
-        name, N, K, wp, ws = layer
-        flexq.linear(self.x[(M, K)], wp, ws, N, GS, ACT_BITS, out=self.y[(M, name)])
+        name, N, K, bits, site, wp, ws = layer
+        flexq.linear(self.x[(M, site)], wp, ws, N, GS, bits, out=self.y[(M, name)])
 
     def run_m(self, M):
         for layer in self.w:
             self.linear(M, layer)
 
-    def step(self):
-        for M in self.ms:
-            self.run_m(M)
-
-    def segments(self, dominant_m):
-        """The step cut into replayable pieces: all layers of an M as one piece,
-        except at the dominant M, where every quantization and every GEMM is
-        its own piece so that events can bracket the GEMM launches."""
+    def segments(self):
+        """The step cut into replayable pieces: at the HBM-bound M all layers
+        of an M are one piece (flexq.linear per layer); at the tensor-bound M
+        every quantization and every GEMM is its own piece so that events can
+        bracket the GEMM launches."""
         segs = []
         for M in self.ms:
-            if M == dominant_m:
+            if self.split_m(M):
                 for layer in self.w:
-                    segs.append(("quant", M, layer[0], (lambda M=M, l=layer: self.quant(M, l))))
-                    segs.append(("gemm", M, layer[0], (lambda M=M, l=layer: self.gemm(M, l))))
+                    segs.append(("quant", M, layer, (lambda M=M, l=layer: self.quant(M, l))))
+                    segs.append(("gemm", M, layer, (lambda M=M, l=layer: self.gemm(M, l))))
             else:
                 segs.append(("all", M, None, (lambda M=M: self.run_m(M))))
         return segs
@@ -336,18 +356,16 @@ def run_flexq(args, rank, world):
     torch.cuda.set_device(device)
     flexq.lib()                                   # fail loudly if not built
     ms, layers = workload_shapes(args.ms, args.layers)
-    dominant_m = max(ms)
     W = Layers(ms, layers, device)
     ops = step_ops(ms, layers)
-    nlay = len(layers)
 
     # eager warm-up (first calls set kernel attributes; nothing is captured yet)
-    for _ in range(2):
-        W.step()
+    for M in ms:
+        W.run_m(M)
     torch.cuda.synchronize(device)
 
     stream = torch.cuda.Stream(device)
-    segs = W.segments(dominant_m)
+    segs = W.segments()
     runners = []
     if args.graph:
         for (_, _, _, fn) in segs:
@@ -399,18 +417,8 @@ def run_flexq(args, rank, world):
     if status != flexq.FLEXQ_OK:
         raise RuntimeError(f"device status after the timed region: {msg}")
 
-    # per-M times and the dominant GEMM launches, from the timed steps' events
-    per_m_ms = []
-    for M in ms:
-        ks = [k for k, sg in enumerate(segs) if sg[1] == M]
-        per_m_ms.append(statistics.mean(evs[i][ks[0]].elapsed_time(evs[i][ks[-1] + 1])
-                                        for i in range(args.steps)))
-    gk = [k for k, sg in enumerate(segs) if sg[0] == "gemm"]
-    dom_durs = [evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps) for k in gk]
-    dom_flops_per_step = sum(2.0 * dominant_m * N * K for (_, N, K) in layers)
-    dom_avg_ms = statistics.mean(dom_durs)
-    dom_flops_per_launch = dom_flops_per_step / nlay
-    achieved_tops = dom_flops_per_launch / (dom_avg_ms / 1e3) / 1e12
+    def seg_ms(k):
+        return statistics.mean(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps))
 
     peaks, peak_src = measured_peaks()
     long_region = elapsed_ms > 1000.0
@@ -419,11 +427,36 @@ def run_flexq(args, rank, world):
     int8_peak = bf16 * INT8_OVER_BF16
     hbm = peaks["hbm_gbs"]
 
+    # per M: device time of its pieces, TOPS, and the GEMM launches alone
     per_m = []
-    for mi, M in enumerate(ms):
-        m_ops = sum(2.0 * M * N * K for (_, N, K) in layers)
-        per_m.append({"M": M, "ms": round(per_m_ms[mi], 5),
-                      "tops": round(m_ops / (per_m_ms[mi] / 1e3) / 1e12, 3)})
+    gemm_ops = gemm_ms = 0.0
+    dec_bytes = dec_ms = 0.0
+    for M in ms:
+        ks = [k for k, sg in enumerate(segs) if sg[1] == M]
+        m_ms = statistics.mean(evs[i][ks[0]].elapsed_time(evs[i][ks[-1] + 1])
+                               for i in range(args.steps))
+        m_ops = sum(2.0 * M * l[1] * l[2] for l in layers)
+        row = {"M": M, "ms": round(m_ms, 5), "tops": round(m_ops / (m_ms / 1e3) / 1e12, 3)}
+        gk = [k for k in ks if segs[k][0] == "gemm"]
+        if gk:
+            g_ms = sum(seg_ms(k) for k in gk)
+            row["gemm_ms"] = round(g_ms, 5)
+            row["gemm_tops"] = round(m_ops / (g_ms / 1e3) / 1e12, 3)
+            row["gemm_frac_int8"] = round(m_ops / (g_ms / 1e3) / 1e12 / int8_peak, 4)
+            row["gemm_us_by_layer"] = {segs[k][2][0]: round(seg_ms(k) * 1e3, 2) for k in gk}
+            gemm_ops += m_ops
+            gemm_ms += g_ms
+        if M <= DECODE_MAX_M:
+            nbytes = sum(linear_bytes(M, l[1], l[2]) for l in layers)
+            gbs = nbytes / (m_ms / 1e3) / 1e9
+            row["GB/s"] = round(gbs, 1)
+            row["frac_hbm"] = round(gbs / hbm, 4)
+            dec_bytes += nbytes
+            dec_ms += m_ms
+        per_m.append(row)
+    achieved_tops = gemm_ops / (gemm_ms / 1e3) / 1e12 if gemm_ms else 0.0
+    n_gemm = sum(1 for sg in segs if sg[0] == "gemm")
+    dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9 if dec_ms else 0.0
 
     # GEMM-only diagnostics per M (after the timed region, not part of value)
     diag = gemm_diagnostics(W, device, hbm, int8_peak) if args.diag else None
@@ -444,38 +477,50 @@ def run_flexq(args, rank, world):
         "data": "synthetic",
         "config": {
             "workload": workload_name(ms, layers),
-            "group_size": GS, "act_bits": ACT_BITS, "weight_bits": 6,
-            "shapes": [[n, N, K] for n, N, K in layers], "M": ms,
+            "group_size": GS, "weight_bits": 6,
+            "act_bits": {l[0]: l[3] for l in layers},
+            "shapes": [[l[0], l[1], l[2]] for l in layers], "M": ms,
             "ops_per_step": ops,
-            "l2": "inputs larger than L2: each step streams 151 MB of distinct packed weights",
+            "l2": (f"inputs larger than L2: each M streams {W.packed_bytes() / 1e6:.0f} MB of "
+                   "distinct packed weights"),
             "timing": "CUDA-graph replay of each step" if args.graph else "eager launches",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
         },
         "per_m": per_m,
         "roofline": {
             "bound": "tensor",
-            "kernel": f"gemm_w6ax_kernel (M={dominant_m} launches)",
+            "kernel": (f"gemm_w6ax GEMM launches at M >= {TENSOR_MIN_M} "
+                       f"({n_gemm} per step)"),
             "achieved": round(achieved_tops, 2),
             "peak": round(int8_peak, 1),
             "unit": "TFLOP/s",
-            "frac": round(achieved_tops / int8_peak, 4),
+            "frac": round(achieved_tops / int8_peak, 4) if int8_peak else None,
             "peak_source": (f"{peak_src}: {'sustained' if long_region else 'burst'} bf16 x "
                             f"{INT8_OVER_BF16:g} (nominal int8/bf16 dense ratio)"),
-            "avg_launch_us": round(dom_avg_ms * 1e3, 2),
+            "avg_launch_us": round(gemm_ms * 1e3 / max(1, n_gemm), 2),
             "traffic": traffic,
+            "decode": {
+                "bound": "hbm",
+                "kernel": f"whole layers (quantization + GEMM) at M <= {DECODE_MAX_M}",
+                "achieved": round(dec_gbs, 1), "peak": round(hbm, 1), "unit": "GB/s",
+                "frac": round(dec_gbs / hbm, 4),
+                "bytes": "0.75 B per weight element + FP16 weight scales + FP16 input and output",
+                "peak_source": f"{peak_src}: copy bandwidth",
+            },
         },
         "gpu_launches": W.launches_per_step() * args.steps,
         "clocks": clock_summary,
     }
     if args.graph:
-        result["config"]["timing"] = ("CUDA-graph replay: one graph per M, one per launch at "
-                                      f"M={dominant_m}; events between graph launches")
+        result["config"]["timing"] = (f"CUDA-graph replay: one graph per M below {TENSOR_MIN_M}, "
+                                      "one per launch above; events between graph launches")
     if diag:
         result["gemm_by_m"] = diag
     if args.diag and rank == 0:
-        result["int8_library_context"] = int8_library_context(W, device, dominant_m)
+        result["int8_library_context"] = int8_library_context(W, device, max(ms))
         result["act_quant"] = act_quant_diagnostics(device, hbm)
         result["mixed_stack"] = stack_diagnostics(device, hbm, int8_peak)
+        result["other_configs"] = run_sweep(device, hbm, int8_peak, subset=True)
     if args.e2e:
         result["e2e"] = run_e2e(W, args, device, world)
     if rank == 0 and world == 1 and args.cpu_baseline:
@@ -524,16 +569,15 @@ def _graph_time_us(body, device, stream, reps):
     return t_us
 
 
-def gemm_diagnostics(W, device, hbm_gbs, int8_peak_tops, reps=10):
+def gemm_diagnostics(W, device, hbm_gbs, int8_peak_tops, reps=None):
     """Per-M times and fractions of the attainable roofline (min(int8 peak,
-    HBM x intensity): HBM-bound at decode sizes, tensor-bound at M = 256 and
-    above) of the seven layers, each timed from a CUDA graph that holds `reps`
-    rounds of them back to back (the other layers' weights stream in between,
-    so each launch reads its weights cold); events bracket the graph replay,
-    so host launch work is not timed.  `gemm_*`: the GEMM alone on quantized
-    activations; `linear_*`: the whole layer from FP16 activations through
-    flexq.linear (one launch with quantization inside the GEMM for batches of
-    at most 2 tokens, the quantizer and the GEMM otherwise)."""
+    HBM x intensity): HBM-bound at decode sizes, tensor-bound at M = 512 and
+    above) of the step's layers, each timed from a CUDA graph that holds
+    `reps` rounds of them back to back (the other layers' weights stream in
+    between, so each launch reads its weights cold); events bracket the graph
+    replay, so host launch work is not timed.  `gemm_*`: the GEMM alone on
+    quantized activations; `linear_*`: the whole layer from FP16 activations
+    through flexq.linear."""
     import torch
     from bit_group_quantized_flexq_b200 import flexq
     out = []
@@ -541,22 +585,22 @@ def gemm_diagnostics(W, device, hbm_gbs, int8_peak_tops, reps=10):
     for M in W.ms:
         for layer in W.w:
             W.quant(M, layer)                     # the GEMM's quantized inputs
+        n_reps = reps or (2 if M >= 4096 else 5)
 
         def gemm_body():
-            for (name, N, K, wp, ws) in W.w:
-                flexq.gemm(W.xq[(M, K)], W.xs[(M, K)], wp, ws, N, GS, ACT_BITS,
-                           out=W.y[(M, name)])
+            for layer in W.w:
+                W.gemm(M, layer)
 
         def linear_body():
             for layer in W.w:
                 W.linear(M, layer)
 
-        t_us = _graph_time_us(gemm_body, device, stream, reps)
-        l_us = _graph_time_us(linear_body, device, stream, reps)
-        flops = sum(2.0 * M * N * K for (_, N, K, _, _) in W.w)
+        t_us = _graph_time_us(gemm_body, device, stream, n_reps)
+        l_us = _graph_time_us(linear_body, device, stream, n_reps)
+        flops = sum(2.0 * M * l[1] * l[2] for l in W.w)
         row = {"M": M}
-        for key, us, nbytes in (("gemm", t_us, sum(gemm_bytes(M, N, K) for (_, N, K, _, _) in W.w)),
-                                ("linear", l_us, sum(linear_bytes(M, N, K) for (_, N, K, _, _) in W.w))):
+        for key, us, nbytes in (("gemm", t_us, sum(gemm_bytes(M, l[1], l[2]) for l in W.w)),
+                                ("linear", l_us, sum(linear_bytes(M, l[1], l[2]) for l in W.w))):
             gbs = nbytes / (us * 1e-6) / 1e9
             tops = flops / (us * 1e-6) / 1e12
             bound, frac = roofline(flops, nbytes, us, hbm_gbs, int8_peak_tops)
@@ -565,7 +609,7 @@ def gemm_diagnostics(W, device, hbm_gbs, int8_peak_tops, reps=10):
             row[f"{key}_GB/s"] = round(gbs, 1)
             row[f"{key}_TOPS"] = round(tops, 2)
             row[f"{key}_frac"] = round(frac, 4)
-        row["plan"] = [list(flexq.plan(M, N, K, GS)) for (_, N, K, _, _) in W.w]
+        row["plan"] = [list(flexq.plan(M, l[1], l[2], GS)) for l in W.w]
         out.append(row)
     return out
 
@@ -607,10 +651,11 @@ def act_quant_diagnostics(device, hbm_gbs, K=8192, ms=(1, 2048, 16384), reps=20)
     return out
 
 
-def stack_diagnostics(device, hbm_gbs, int8_peak_tops, ms=(1, 16, 512, 8192)):
+def stack_diagnostics(device, hbm_gbs, int8_peak_tops, ms=(1, 16)):
     """The mixed W6A6/W6A8 layer stack (stack.LayerStack) on one LLaMA-2-70B
     block (q, k, v, o, gate, up, down; 8-bit activations for down), seeded
-    synthetic weights drawn on the device: per M, the device time of one
+    synthetic weights drawn on the device, at the decode sizes (the step
+    above measures the large ones): per M, the device time of one
     block forward from FP16 activations (CUDA graph of a few forwards), with
     the attainable roofline min(int8 peak, HBM x intensity); once with
     every layer its own GEMM, once with q/k/v and gate/up merged
@@ -655,7 +700,7 @@ def _stack_rows(st, device, hbm_gbs, int8_peak_tops, ms):
     return rows
 
 
-def run_sweep(device, hbm_gbs, int8_peak_tops):
+def run_sweep(device, hbm_gbs, int8_peak_tops, subset=False):
     """The other measured configurations, one JSON line (`--sweep`; not part
     of the default run): the LLaMA-2-13B W6A8 layers at M in {1, 64, 4096}
     and the N = K = 8192 sweep over group size {32, 64, 128, 256}, W6A6 and
@@ -663,7 +708,9 @@ def run_sweep(device, hbm_gbs, int8_peak_tops):
     (codes given) and the whole layer from FP16 activations (flexq.linear),
     device time per call from a CUDA graph that rotates over enough copies
     of the packed weights to exceed L2, against the attainable rate
-    min(int8 peak, HBM bandwidth x arithmetic intensity)."""
+    min(int8 peak, HBM bandwidth x arithmetic intensity).  With subset=True
+    (the default run's extra key): the 13B layers at all their M, and the
+    sweep at M in {1, 4096} for every group size, W6A6 and W6A8."""
     import torch
     from bit_group_quantized_flexq_b200 import flexq, inputs
     stream = torch.cuda.Stream(device)
@@ -711,10 +758,11 @@ def run_sweep(device, hbm_gbs, int8_peak_tops):
             out["13b_w6a8"].append(case(M, N, K, 128, 8, wp, ws, copies))
         del copies
         torch.cuda.empty_cache()
+    sweep_m = (1, 4096) if subset else tuple(inputs.SWEEP_M)
     for gs in (32, 64, 128, 256):
         wp, ws, copies = weights(8192, 8192, gs, 0.02)
         for bits in (6, 8):
-            for M in (1, 8, 32, 128, 1024, 4096, 16384):
+            for M in sweep_m:
                 out["sweep_8192"].append(case(M, 8192, 8192, gs, bits, wp, ws, copies))
         del copies
         torch.cuda.empty_cache()
@@ -746,7 +794,7 @@ def int8_library_context(W, device, M, reps=20):
 
     try:
         shapes = []
-        for (name, N, K, _, _) in W.w:
+        for (name, N, K, _, _, _, _) in W.w:
             us, tops = time_mm(M, N, K)
             shapes.append({"layer": name, "M": M, "N": N, "K": K, "us": us, "TOPS": tops})
         us, tops = time_mm(8192, 8192, 8192)
@@ -767,9 +815,9 @@ def run_e2e(W, args, device, world):
     import torch
     from bit_group_quantized_flexq_b200 import flexq
     keys = [(M, layer) for M in W.ms for layer in W.w]
-    hx = {(M, l[0]): W.x[(M, l[2])].cpu().pin_memory() for M, l in keys}
+    hx = {(M, l[0]): W.x[(M, l[4])].cpu().pin_memory() for M, l in keys}
     hy = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in W.y.items()}
-    dx = {(M, l[0]): torch.empty_like(W.x[(M, l[2])]) for M, l in keys}
+    dx = {(M, l[0]): torch.empty_like(W.x[(M, l[4])]) for M, l in keys}
     h2d = sum(v.numel() * 2 for v in hx.values())
     d2h = sum(v.numel() * 2 for v in W.y.values())
     s_in, s_c, s_out = (torch.cuda.Stream(device) for _ in range(3))
@@ -780,7 +828,7 @@ def run_e2e(W, args, device, world):
     started = [False]
 
     def step():
-        for M, (name, N, K, wp, ws) in keys:
+        for M, (name, N, K, bits, site, wp, ws) in keys:
             k = (M, name)
             if started[0]:
                 s_in.wait_event(done_c[k])        # the previous step's layer has read dx
@@ -791,7 +839,7 @@ def run_e2e(W, args, device, world):
             if started[0]:
                 s_c.wait_event(done_out[k])       # the previous step's copy out has read y
             with torch.cuda.stream(s_c):
-                flexq.linear(dx[k], wp, ws, N, GS, ACT_BITS, out=W.y[k])
+                flexq.linear(dx[k], wp, ws, N, GS, bits, out=W.y[k])
                 done_c[k].record(s_c)
             s_out.wait_event(done_c[k])
             with torch.cuda.stream(s_out):
@@ -819,7 +867,7 @@ def run_e2e(W, args, device, world):
     t1.record(main)
     torch.cuda.synchronize(device)
     t_max = max_over_ranks(t0.elapsed_time(t1) / 1e3, device)
-    ops = step_ops(W.ms, [(n, N, K) for (n, N, K, _, _) in W.w])
+    ops = step_ops(W.ms, W.layers)
     return {"value": round(aggregate(ops * args.steps, world, t_max) / 1e12, 3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(t_max * 1e3 / args.steps, 4),
@@ -827,66 +875,108 @@ def run_e2e(W, args, device, world):
 
 
 # ------------------------------------------------------- CPU oracle arm ----
-def oracle_sample_layers():
-    """A bounded sample of the workload for the CPU oracle: the M = 1 and
-    M = 16 rows of the step over all seven layers."""
-    from bit_group_quantized_flexq_b200 import inputs
-    return [1, 16], list(inputs.LLAMA2_7B_LAYERS)
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 class OracleSample:
-    def __init__(self):
+    """A bounded sample of the step for the CPU oracle: for every M of the
+    step, `rows` seeded rows of that M's activations (all of them where M is
+    smaller) through all five layers.  The oracle's cost is linear in the
+    rows, so a larger M's time is the sample's time scaled by M / rows
+    (extrapolated); the weights are quantized once, outside the timing, as
+    the method does offline."""
+
+    def __init__(self, rows=1):
         from bit_group_quantized_flexq_b200 import inputs
         from oracle import flexq_oracle as orc
         self.orc = orc
-        self.ms, self.layers = oracle_sample_layers()
+        self.ms, self.layers = workload_shapes()
+        self.rows = rows
         self.w = []
-        for name, N, K in self.layers:
-            w16 = inputs.weights(N, K, std=0.02, seed=inputs.layer_seed("7b", name)).numpy()
+        for name, N, K, bits, site in self.layers:
+            w16 = inputs.weights(N, K, std=WEIGHT_STD,
+                                 seed=inputs.layer_seed("70b", name)).numpy()
             qw, sw = orc.quantize_weight(w16, GS)      # offline step, not timed
-            self.w.append((name, N, K, qw, sw))
-        self.x = {(M, K): inputs.activations(M, K, outlier_frac=0.01, outlier_scale=20.0,
-                                             seed=inputs.layer_seed("7b-x", M, K)).numpy()
-                  for M in self.ms for K in {K for (_, _, K) in self.layers}}
-        self.ops = step_ops(self.ms, self.layers)
-
-    def step(self):
-        orc = self.orc
+            self.w.append((name, N, K, bits, site, qw, sw))
+        self.x = {}
         for M in self.ms:
-            for (name, N, K, qw, sw) in self.w:
-                qa, sa = orc.quantize_act(self.x[(M, K)], GS, ACT_BITS)
-                orc.to_fp16(orc.gemm_fp64(qa, sa, qw, sw, GS))
+            r = min(M, rows)
+            for site, K in {l[4]: l[2] for l in self.layers}.items():
+                x = inputs.activations(r, K, outlier_frac=OUTLIER_FRAC,
+                                       outlier_scale=OUTLIER_SCALE,
+                                       seed=inputs.layer_seed("70b-x-cpu", M, site))
+                self.x[(M, site)] = x.numpy()
+        self.jobs = [(M, l) for M in self.ms for l in self.w]
+        # operations the sample computes, and those of the M it stands for
+        self.ops_sample = sum(2.0 * min(M, rows) * l[1] * l[2] for M, l in self.jobs)
+        self.ops_full = step_ops(self.ms, self.layers)
+
+    def job(self, item):
+        M, (name, N, K, bits, site, qw, sw) = item
+        orc = self.orc
+        qa, sa = orc.quantize_act(self.x[(M, site)], GS, bits)
+        orc.to_fp16(orc.gemm_fp64(qa, sa, qw, sw, GS))
+
+    def step(self, threads=1):
+        if threads <= 1:
+            for item in self.jobs:
+                self.job(item)
+            return
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(self.job, self.jobs))
 
 
-def run_cpu_baseline(budget_s=20.0):
-    s = OracleSample()
+def run_cpu_baseline(budget_s=30.0):
+    """The oracle on the host cores: one pass of the sample on one thread and
+    passes on every core (numpy releases the GIL inside its array loops, so
+    threads run the (M, layer) jobs in parallel)."""
+    s = OracleSample(rows=1)
+    cores = os.cpu_count() or 1
     t0 = time.perf_counter()
-    n = 0
+    s.step(1)
+    dt1 = time.perf_counter() - t0
+    n, t0 = 0, time.perf_counter()
     while True:
-        s.step()
+        s.step(cores)
         n += 1
-        if time.perf_counter() - t0 > budget_s / 2 or n >= 3:
+        if time.perf_counter() - t0 > budget_s / 3 or n >= 3:
             break
-    dt = (time.perf_counter() - t0) / n
-    return {"value": round(s.ops / dt / 1e12, 9), "unit": UNIT, "cores": 1,
-            "kind": "oracle",
-            "sample": (f"oracle (numpy, int64 group dot products + FP64 rescale) on M in "
-                       f"{s.ms} over all seven LLaMA-2-7B layers; {n} passes of "
-                       f"{dt:.2f} s; integer matmul runs on one thread")}
+    dtn = (time.perf_counter() - t0) / n
+    return {"value": round(s.ops_sample / dtn / 1e12, 9), "unit": UNIT, "cores": cores,
+            "kind": "oracle", "cpu_model": cpu_model(),
+            "one_thread": {"value": round(s.ops_sample / dt1 / 1e12, 9), "cores": 1},
+            "step_s_extrapolated": round(dtn * s.ops_full / s.ops_sample, 1),
+            "sample": (f"oracle (numpy: int64 group dot products + FP64 rescale, activation "
+                       f"quantization included) on one seeded row of each M in {s.ms} through "
+                       f"all five layers ({s.ops_sample / 1e9:.1f} GOP); {n} passes of "
+                       f"{dtn:.2f} s on {cores} threads, {dt1:.2f} s on one; the whole step "
+                       f"scales linearly in the rows (extrapolated)")}
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    s = OracleSample()
+    s = OracleSample(rows=1)
+    cores = os.cpu_count() or 1
     for _ in range(args.warmup):
-        s.step()
+        s.step(cores)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        s.step()
+        s.step(cores)
     dt = time.perf_counter() - t0
-    value = s.ops * args.steps / dt / 1e12
+    value = s.ops_sample * args.steps / dt / 1e12
     ms, layers = workload_shapes()
+    sample = (f"each step: one seeded row of each M in {s.ms} through all five layers "
+              f"({s.ops_sample / 1e9:.1f} GOP), on {cores} threads")
     out = {
         "impl": "reference",
         "metric": METRIC, "value": round(value, 9), "unit": UNIT, "n_gpus": world,
@@ -894,10 +984,9 @@ def run_reference(args, rank, world):
         "ms_per_step": round(dt * 1e3 / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int64", "data": "synthetic",
-        "config": {"workload": workload_name(ms, layers),
-                   "sample": f"each step: M in {s.ms} over all seven layers"},
-        "cpu_baseline": {"value": round(value, 9), "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"M in {s.ms} over all seven layers per step"},
+        "config": {"workload": workload_name(ms, layers), "sample": sample},
+        "cpu_baseline": {"value": round(value, 9), "unit": UNIT, "cores": cores,
+                         "kind": "oracle", "cpu_model": cpu_model(), "sample": sample},
         "e2e": {"value": round(value, 9), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -919,7 +1008,7 @@ def parse_args(argv=None):
     p.add_argument("--no-e2e", dest="e2e", action="store_false")
     p.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     p.add_argument("--no-diag", dest="diag", action="store_false")
-    p.add_argument("--cpu-budget-s", type=float, default=20.0)
+    p.add_argument("--cpu-budget-s", type=float, default=30.0)
     p.add_argument("--sweep", action="store_true",
                    help="measure the 13B W6A8 layers and the N = K = 8192 group-size sweep "
                         "instead of the step (one JSON line)")

@@ -662,6 +662,11 @@ int flexq_gemm_static_scratch(int M, int N, int K, int group_size, int act_bits,
   int rc = check_gemm_shape(M, N, K, group_size);
   if (rc) return rc;
   if (M == 0) return ok();
+  // every pointer is checked before anything is enqueued (the counter clear
+  // below is the first work on the stream)
+  const void* ptrs[] = {Xq, X_scales, Wq_packed, W_scales, Y_fp16};
+  const char* names[] = {"Xq", "X_scales", "Wq_packed", "W_scales", "Y"};
+  if ((rc = check_ptrs(5, ptrs, names))) return rc;
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
   const size_t need = workspace_bytes_for(make_plan(M, N, K, group_size, st->sms, false), M, N);

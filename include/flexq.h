@@ -236,9 +236,11 @@ int flexq_linear_w6a8(int M, int N, int K, int group_size, const void* X_fp16,
  *   allocates nothing (no cudaMalloc, cudaFree or allocating library call).
  *   Shapes whose plan needs more split-K scratch than 16 MiB are rejected
  *   with FLEXQ_ERR_UNSUPPORTED (no plan the library picks by itself does).
- *   The first call on a device looks up the scratch's device address; make
- *   that first call before capturing a stream.  Each call first clears the
- *   scratch's arrival counters on `stream` (a 4 KB memset), then launches.
+ *   Shapes and pointers are checked first; an invalid argument returns its
+ *   status with nothing enqueued.  The first call on a device looks up the
+ *   scratch's device address; make that first call before capturing a
+ *   stream.  Each call then clears the scratch's arrival counters on
+ *   `stream` (a 4 KB memset) and launches.
  *   All calls on a device share the one scratch, which keeps the last call's
  *   partial tiles: two calls that overlap on the GPU (different streams, or
  *   concurrently running graphs) race on it and give wrong results.

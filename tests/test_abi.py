@@ -161,3 +161,20 @@ def test_linear_workspace_layout(L):
     assert flexq.linear_workspace_bytes(4, 200, 4096, 128) == 0
     assert flexq.linear_launches(0, 4096, 4096, 128) == 0
     assert L.flexq_debug_force_linear_route(3) == flexq.FLEXQ_ERR_INVALID_ARG
+
+
+def test_static_scratch_validation_before_any_launch(L):
+    f = L.flexq_gemm_static_scratch
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, NULL)
+    assert f(4, 256, 256, 128, 7, *args) == flexq.FLEXQ_ERR_INVALID_ARG       # act_bits
+    assert b"act_bits" in L.flexq_last_error_message()
+    assert f(4, 200, 256, 128, 6, *args) == flexq.FLEXQ_ERR_UNSUPPORTED       # N % 128
+    assert f(4, 256, 256, 48, 8, *args) == flexq.FLEXQ_ERR_UNSUPPORTED        # group size
+    assert f(4, 256, 384, 256, 6, *args) == flexq.FLEXQ_ERR_UNSUPPORTED       # K % 256
+    assert f(-1, 256, 256, 128, 6, *args) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert f(0, 256, 256, 128, 6, *args) == flexq.FLEXQ_OK                    # empty batch
+    # pointers are checked before the counter clear is enqueued: no GPU needed
+    assert f(4, 256, 256, 128, 6, FAKE, NULL, FAKE, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert b"X_scales" in L.flexq_last_error_message()
+    assert f(4, 256, 256, 128, 8, FAKE, FAKE, FAKE, FAKE, MISALIGNED, NULL) == \
+        flexq.FLEXQ_ERR_MISALIGNED

@@ -86,3 +86,14 @@ def test_roofline_picks_the_lower_bound():
     bound, frac = bench.roofline(ops, bench.gemm_bytes(2048, 4096, 4096), 100.0, 6500.0, 3300.0)
     assert bound == "tensor"
     assert abs(frac - ops / 100e-6 / 1e12 / 3300.0) < 1e-9
+
+
+def test_headline_workload_is_the_llama2_70b_configuration():
+    ms, layers = bench.workload_shapes()
+    assert ms == [1, 16, 512, 8192]
+    assert [(n, N, K, b) for (n, N, K, b, _) in layers] == [
+        ("q", 8192, 8192, 6), ("o", 8192, 8192, 6), ("gate", 28672, 8192, 6),
+        ("up", 28672, 8192, 6), ("down", 8192, 28672, 8)]
+    # gate and up read the same input; every other layer its own
+    assert len({site for (*_, site) in layers}) == 4
+    assert "LLaMA-2-70B" in bench.workload_name(ms, layers)

@@ -160,6 +160,34 @@ def test_full_size_sampled_rows(M, N, K, gs, bits, std, frac, scale):
     assert_within(y[rows], y64, TOL)
 
 
+# the LLaMA-2-70B layers of the headline step at every one of its M: one weight
+# draw per shape (quantized by the GPU and by the oracle once), sampled rows
+_70B = {}
+
+
+def _70b_layer(N, K):
+    if (N, K) not in _70B:
+        seed = inputs.layer_seed("full70", N, K)
+        w = inputs.weights(N, K, std=0.015, seed=seed)
+        wp, ws = flexq.quantize_weight(w.cuda(), 128)
+        qw, sw = orc.quantize_weight(w.numpy(), 128)
+        _70B.clear()
+        _70B[(N, K)] = (wp, ws, qw, sw)
+    return _70B[(N, K)]
+
+
+@pytest.mark.parametrize("M", [1, 16, 512, 8192])
+@pytest.mark.parametrize("N,K,bits", [(28672, 8192, 6), (8192, 8192, 6), (8192, 28672, 8)])
+def test_llama2_70b_layers_sampled_rows(N, K, bits, M):
+    wp, ws, qw, sw = _70b_layer(N, K)
+    x = inputs.activations(M, K, outlier_frac=0.005, outlier_scale=50.0,
+                           seed=inputs.layer_seed("full70-x", M, N, K))
+    y = np16(flexq.linear(x.cuda(), wp, ws, N, 128, bits))
+    rows = sorted(set(np.random.default_rng(M + N).integers(0, M, 5).tolist()) | {0, M - 1})
+    qa, sa = orc.quantize_act(x.numpy()[rows], 128, bits)
+    assert_within(y[rows], orc.gemm_fp64(qa, sa, qw, sw, 128), TOL)
+
+
 # ------------------------------------------------------ bounded waits ------
 def test_stalled_pipeline_reports_timeout_and_context_survives():
     M, N, K, gs = 16, 256, 1024, 128
