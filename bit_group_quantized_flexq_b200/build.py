@@ -13,7 +13,8 @@ ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "flexq_api.cu")
 LIB = os.path.join(PKG, "libflexq.so")
 DEPS = [os.path.join(PKG, "csrc", f) for f in
-        ("flexq_api.cu", "flexq_gemm.cuh", "flexq_quant.cuh", "flexq_ptx.cuh")] + \
+        ("flexq_api.cu", "flexq_gemm.cuh", "flexq_gemm_wide.cuh", "flexq_quant.cuh",
+                  "flexq_ptx.cuh")] + \
        [os.path.join(ROOT, "include", "flexq.h")]
 
 NVCC_FLAGS = [

@@ -17,6 +17,7 @@
 
 #include "../../include/flexq.h"
 #include "flexq_gemm.cuh"
+#include "flexq_gemm_wide.cuh"
 #include "flexq_quant.cuh"
 
 namespace {
@@ -131,7 +132,7 @@ int max_split_for(int T) {
     case 16: return flexq::GemmCfg<16>::kMaxSplit;
     case 32: return flexq::GemmCfg<32>::kMaxSplit;
     case 64: return flexq::GemmCfg<64>::kMaxSplit;
-    default: return flexq::GemmCfg<128>::kMaxSplit;
+    default: return flexq::WideCfg::kMaxSplit;
   }
 }
 
@@ -145,7 +146,7 @@ int min_blocks_for(int T) {
     case 16: return flexq::GemmCfg<16>::kMinBlocks;
     case 32: return flexq::GemmCfg<32>::kMinBlocks;
     case 64: return flexq::GemmCfg<64>::kMinBlocks;
-    default: return flexq::GemmCfg<128>::kMinBlocks;
+    default: return 1;                       // the wide kernel: one CTA per SM
   }
 }
 
@@ -320,6 +321,50 @@ int launch_gemm_t(DeviceState* st, const CUtensorMap& map, const CUtensorMap& ma
   return FLEXQ_OK;
 }
 
+// 128-token tiles: the warpgroup-role kernel of flexq_gemm_wide.cuh.
+template <bool PARTIALS>
+int launch_gemm_wide(DeviceState* st, const CUtensorMap& map, flexq::GemmArgs a,
+                     long long grid_ctas, cudaStream_t stream) {
+  using Cfg = flexq::WideCfg;
+  auto kern = flexq::gemm_w6ax_wide_kernel<PARTIALS>;
+  const unsigned bit = 1u << (12 + (PARTIALS ? 1 : 0));
+  const int ctrl_off = (Cfg::kMainBytes + 15) & ~15;
+  const int smem = 1024 + ctrl_off + static_cast<int>(sizeof(flexq::WideCtrl));
+  {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!(st->attr_mask & bit)) {
+      // the warpgroups' register budgets must fit in what the CTA launches
+      // with, or the epilogue's increase would wait for registers that never
+      // come: refuse to launch instead
+      cudaFuncAttributes fa;
+      cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+      const long long launch_regs = static_cast<long long>(fa.numRegs) * Cfg::kThreads;
+      const long long budget = 128LL * Cfg::kRegsCtl + 128LL * Cfg::kRegsUnpack + 256LL * Cfg::kRegsEpi;
+      if (launch_regs < budget)
+        return fail(FLEXQ_ERR_CUDA, "wide GEMM compiled with %d registers per thread; its register "
+                    "split needs %lld per CTA", fa.numRegs, budget);
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+      st->attr_mask |= bit;
+    }
+  }
+  a.ctrl_offset = ctrl_off;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid_ctas), 1, 1);
+  cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map, a);
+  if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
+  return FLEXQ_OK;
+}
+
 // The caller's split-K workspace against the plan: none (NULL, 0 bytes)
 // runs every tile whole; one too small for the plan is an error.
 int apply_workspace(Plan* plan, int M, int N, void* workspace, size_t workspace_bytes) {
@@ -375,6 +420,9 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
   a.wp = static_cast<const uint8_t*>(Wp);
   a.y = static_cast<__half*>(Y);
   a.p = P;
+  a.sa = static_cast<const __half*>(Xs);
+  a.sw = static_cast<const __half*>(Ws);
+  a.sa_ld = act_scales_ld(M);
   if (plan.split > 1) {
     a.ws_cnt = static_cast<unsigned int*>(workspace);
     a.ws_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kCounterBytes);
@@ -391,7 +439,7 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
     case 16: rc = partials ? launch_gemm_t<16, true>(st, map, map_sa, map_sw, a, plan.ctas, s) : launch_gemm_t<16, false>(st, map, map_sa, map_sw, a, plan.ctas, s); break;
     case 32: rc = partials ? launch_gemm_t<32, true>(st, map, map_sa, map_sw, a, plan.ctas, s) : launch_gemm_t<32, false>(st, map, map_sa, map_sw, a, plan.ctas, s); break;
     case 64: rc = partials ? launch_gemm_t<64, true>(st, map, map_sa, map_sw, a, plan.ctas, s) : launch_gemm_t<64, false>(st, map, map_sa, map_sw, a, plan.ctas, s); break;
-    default: rc = partials ? launch_gemm_t<128, true>(st, map, map_sa, map_sw, a, plan.ctas, s) : launch_gemm_t<128, false>(st, map, map_sa, map_sw, a, plan.ctas, s); break;
+    default: rc = partials ? launch_gemm_wide<true>(st, map, a, plan.ctas, s) : launch_gemm_wide<false>(st, map, a, plan.ctas, s); break;
   }
   return rc ? rc : ok();
 }

@@ -58,6 +58,9 @@ struct GemmArgs {
   __half* y;               // [M, N] output (GEMM mode)
   int32_t* p;              // [G, M, N] partials (debug mode)
   const __half* x;         // [M, K] FP16 activations (fused quantization only)
+  const __half* sa;        // activation scales [G][sa_ld] (wide kernel)
+  const __half* sw;        // weight scales [G][N] (wide kernel)
+  int sa_ld;
   int qmax;                // activation code range Q (fused quantization only)
   int fq_offset;           // byte offset of the fused quantizer's smem block
   float* ws_part;          // split-K partial tiles [tiles][split][T][128] (split > 1)

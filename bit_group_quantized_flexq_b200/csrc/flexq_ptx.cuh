@@ -290,6 +290,20 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
+// ------------------------------------------------------ register split ----
+// Per-warpgroup register budgets: every warp of a warpgroup executes the same
+// instruction.  A decrease returns registers to the CTA's pool; an increase
+// waits until the pool holds enough, so the budgets of all warpgroups must
+// add up to at most the registers the CTA was launched with.
+template <uint32_t R>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+
 // ------------------------------------------------------------- cluster -----
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

@@ -45,7 +45,7 @@ def _case(M, N, K, gs, bits, seed):
 SEQUENCE = [
     (1, 4096, 4096, 128, 6, 11),      # decode: K split 8 ways through the scratch
     (16, 11008, 4096, 128, 8, 12),    # decode, W6A8, split 3
-    (200, 384, 1024, 64, 6, 13),      # two token tiles
+    (200, 384, 4096, 64, 6, 13),      # two 128-token tiles, split 2
     (1, 4096, 4096, 128, 6, 14),      # the first shape again, new inputs
 ]
 
