@@ -245,7 +245,7 @@ def measured_peaks():
 
 def kernel_source_digest():
     h = hashlib.sha256()
-    for f in ("flexq_gemm.cuh", "flexq_ptx.cuh", "flexq_api.cu"):
+    for f in ("flexq_gemm.cuh", "flexq_gemm_wide.cuh", "flexq_ptx.cuh", "flexq_api.cu"):
         with open(os.path.join(ROOT, "bit_group_quantized_flexq_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -254,7 +254,7 @@ def kernel_source_digest():
 def profiled_traffic():
     """DRAM bytes per launch of the dominant GEMM from the committed ncu
     summary, or None when the kernel source changed since that capture."""
-    p = os.path.join(ROOT, "profiles", "gemm_m2048_traffic.json")
+    p = os.path.join(ROOT, "profiles", "gemm_wide_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
@@ -489,8 +489,8 @@ def run_flexq(args, rank, world):
         "per_m": per_m,
         "roofline": {
             "bound": "tensor",
-            "kernel": (f"gemm_w6ax GEMM launches at M >= {TENSOR_MIN_M} "
-                       f"({n_gemm} per step)"),
+            "kernel": (f"gemm_w6ax_wide_kernel (GEMM launches at M >= {TENSOR_MIN_M}, "
+                       f"{n_gemm} per step)"),
             "achieved": round(achieved_tops, 2),
             "peak": round(int8_peak, 1),
             "unit": "TFLOP/s",
@@ -655,25 +655,25 @@ def stack_diagnostics(device, hbm_gbs, int8_peak_tops, ms=(1, 16)):
     """The mixed W6A6/W6A8 layer stack (stack.LayerStack) on one LLaMA-2-70B
     block (q, k, v, o, gate, up, down; 8-bit activations for down), seeded
     synthetic weights drawn on the device, at the decode sizes (the step
-    above measures the large ones): per M, the device time of one
-    block forward from FP16 activations (CUDA graph of a few forwards), with
-    the attainable roofline min(int8 peak, HBM x intensity); once with
-    every layer its own GEMM, once with q/k/v and gate/up merged
-    (fuse_sites)."""
+    above measures the large ones): per M, the device time of one block
+    forward from FP16 activations (CUDA graph of a few forwards), with the
+    attainable roofline min(int8 peak, HBM x intensity).  Three ways to run
+    it: the layers of one input site as one grouped launch, each with its
+    own packed weights (`by_m`, the default); every layer its own launch
+    (`by_m_single_launches`); the layers of a site merged into one weight
+    matrix (`by_m_fused_sites`, a different weight layout)."""
     import torch
     from bit_group_quantized_flexq_b200 import inputs, stack
     res = {}
-    for fuse in (False, True):
-        st = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED, device=device,
-                              fuse_sites=fuse)
-        res["fused_sites" if fuse else "layers"] = _stack_rows(st, device, hbm_gbs,
-                                                               int8_peak_tops, ms)
+    for key, kw in (("by_m", {}), ("by_m_single_launches", {"group_sites": False}),
+                    ("by_m_fused_sites", {"fuse_sites": True})):
+        st = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED, device=device, **kw)
+        res[key] = _stack_rows(st, device, hbm_gbs, int8_peak_tops, ms)
         bits, gs, packed = st.bits, st.gs, st.packed_bytes()
         del st
         torch.cuda.empty_cache()
     return {"block": "LLaMA-2-70B (q, k, v, o, gate, up, down)",
-            "act_bits": bits, "group_size": gs, "packed_MB": round(packed / 1e6, 1),
-            "by_m": res["layers"], "by_m_fused_sites": res["fused_sites"]}
+            "act_bits": bits, "group_size": gs, "packed_MB": round(packed / 1e6, 1), **res}
 
 
 def _stack_rows(st, device, hbm_gbs, int8_peak_tops, ms):

@@ -286,7 +286,7 @@ int smem_bytes_for() {
 
 template <int T, bool PARTIALS, bool FUSEDQ = false>
 int launch_gemm_t(DeviceState* st, const CUtensorMap& map, const CUtensorMap& map_sa,
-                  const CUtensorMap& map_sw, flexq::GemmArgs a, long long grid_ctas,
+                  const flexq::LayerTable& tab, flexq::GemmArgs a, long long grid_ctas,
                   cudaStream_t stream) {
   using Cfg = flexq::GemmCfg<T>;
   auto kern = flexq::gemm_w6ax_kernel<T, PARTIALS, FUSEDQ>;
@@ -316,9 +316,28 @@ int launch_gemm_t(DeviceState* st, const CUtensorMap& map, const CUtensorMap& ma
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map, map_sa, map_sw, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map, map_sa, tab, a);
   if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
   return FLEXQ_OK;
+}
+
+// The layer table of a launch with one layer.
+flexq::LayerTable single_layer_table(const CUtensorMap& map_sw, const void* Wp, void* Y, int N,
+                                     const Plan& plan) {
+  flexq::LayerTable t;
+  memset(&t, 0, sizeof(t));
+  t.sw[0] = map_sw;
+  t.wp[0] = static_cast<const uint8_t*>(Wp);
+  t.y[0] = static_cast<__half*>(Y);
+  t.part0[0] = 0;
+  t.N[0] = N;
+  t.unit0[0] = 0;
+  t.unit0[1] = static_cast<int>(plan.ctas);
+  t.n_full[0] = static_cast<int>(plan.n_full);
+  t.split[0] = plan.split;
+  t.tile0[0] = 0;
+  t.n_layers = 1;
+  return t;
 }
 
 // 128-token tiles: the warpgroup-role kernel of flexq_gemm_wide.cuh.
@@ -435,10 +454,11 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
   a.split = plan.split;
   a.stall = g_inject_stall.exchange(0);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const flexq::LayerTable tab = single_layer_table(map_sw, Wp, Y, N, plan);
   switch (plan.T) {
-    case 16: rc = partials ? launch_gemm_t<16, true>(st, map, map_sa, map_sw, a, plan.ctas, s) : launch_gemm_t<16, false>(st, map, map_sa, map_sw, a, plan.ctas, s); break;
-    case 32: rc = partials ? launch_gemm_t<32, true>(st, map, map_sa, map_sw, a, plan.ctas, s) : launch_gemm_t<32, false>(st, map, map_sa, map_sw, a, plan.ctas, s); break;
-    case 64: rc = partials ? launch_gemm_t<64, true>(st, map, map_sa, map_sw, a, plan.ctas, s) : launch_gemm_t<64, false>(st, map, map_sa, map_sw, a, plan.ctas, s); break;
+    case 16: rc = partials ? launch_gemm_t<16, true>(st, map, map_sa, tab, a, plan.ctas, s) : launch_gemm_t<16, false>(st, map, map_sa, tab, a, plan.ctas, s); break;
+    case 32: rc = partials ? launch_gemm_t<32, true>(st, map, map_sa, tab, a, plan.ctas, s) : launch_gemm_t<32, false>(st, map, map_sa, tab, a, plan.ctas, s); break;
+    case 64: rc = partials ? launch_gemm_t<64, true>(st, map, map_sa, tab, a, plan.ctas, s) : launch_gemm_t<64, false>(st, map, map_sa, tab, a, plan.ctas, s); break;
     default: rc = partials ? launch_gemm_wide<true>(st, map, a, plan.ctas, s) : launch_gemm_wide<false>(st, map, a, plan.ctas, s); break;
   }
   return rc ? rc : ok();
@@ -532,9 +552,238 @@ int linear_common(int M, int N, int K, int gs, int bits, const void* X, const vo
   a.n_full = static_cast<int>(plan.n_full);
   a.split = plan.split;
   a.stall = g_inject_stall.exchange(0);
-  rc = launch_gemm_t<16, false, true>(st, map_x, map_sa, map_sw, a, plan.ctas,
+  const flexq::LayerTable tab = single_layer_table(map_sw, Wp, Y, N, plan);
+  rc = launch_gemm_t<16, false, true>(st, map_x, map_sa, tab, a, plan.ctas,
                                       static_cast<cudaStream_t>(stream));
   return rc ? rc : ok();
+}
+
+// ------------------------------------------------------ grouped launches --
+// Layers that read the same activations (the q, k and v projections, or gate
+// and up) in one launch of the decode kernel: one set of CTAs for all of
+// them, so that a layer's set-up, first-byte latency and split-K tail overlap
+// the other layers' streaming instead of following it.  Each layer keeps its
+// own packed weights, scales and output.  The token tile follows M as for a
+// single layer; with fewer output tiles in all layers than CTA slots every
+// tile is split along K by the same factor, otherwise nothing is split.
+// Batches that take 128-token tiles run the layers one launch after another.
+struct GroupPlan {
+  int T = 0, split = 1, n = 0;
+  long long tiles[flexq::kMaxLayers] = {};
+  long long n_split[flexq::kMaxLayers] = {};
+  long long ctas = 0;
+  size_t ws_bytes = 0;
+};
+
+GroupPlan make_group_plan(int M, const int* N, int n, int K, int gs, int sms,
+                          bool allow_split = true) {
+  GroupPlan g;
+  g.n = n;
+  long long n_sum = 0;
+  for (int l = 0; l < n; ++l) n_sum += N[l];
+  g.T = make_plan(M, static_cast<int>(std::min<long long>(n_sum, 1 << 30)), K, gs, sms, false).T;
+  const long long mtiles = (M + g.T - 1) / g.T;
+  long long total = 0;
+  for (int l = 0; l < n; ++l) total += (g.tiles[l] = static_cast<long long>(N[l] / 128) * mtiles);
+  const long long slots = static_cast<long long>(sms) * min_blocks_for(g.T);
+  const long long max_s = std::min<long long>(max_split_for(g.T), K / 256);
+  long long s = total < slots ? slots / total : 1;
+  const int fS = g_force_split.load();
+  if (fS >= 1 && fS <= max_split_for(g.T) && fS <= K / 256) s = fS;
+  s = std::max<long long>(1, std::min(s, max_s));
+  if (!allow_split || (s > 1 && total > kMaxSplitTiles)) s = 1;
+  g.split = static_cast<int>(s);
+  size_t part = 0;
+  for (int l = 0; l < n; ++l) {
+    g.n_split[l] = s > 1 ? g.tiles[l] : 0;
+    g.ctas += (g.tiles[l] - g.n_split[l]) + g.n_split[l] * s;
+    part += static_cast<size_t>(g.n_split[l]) * s * g.T * 128 * sizeof(float);
+  }
+  g.ws_bytes = s > 1 ? kCounterBytes + part : 0;
+  return g;
+}
+
+int check_group(int M, int K, int gs, int bits, int n_layers, const flexq_layer_t* layers,
+                int* N) {
+  if (bits != 6 && bits != 8) return fail(FLEXQ_ERR_INVALID_ARG, "act_bits=%d is not 6 or 8", bits);
+  if (n_layers < 1 || n_layers > flexq::kMaxLayers)
+    return fail(FLEXQ_ERR_INVALID_ARG, "n_layers=%d not in 1..%d", n_layers, flexq::kMaxLayers);
+  if (!layers) return fail(FLEXQ_ERR_INVALID_ARG, "layers is NULL");
+  for (int l = 0; l < n_layers; ++l) {
+    int rc = check_gemm_shape(M, layers[l].N, K, gs);
+    if (rc) return rc;
+    N[l] = layers[l].N;
+  }
+  return FLEXQ_OK;
+}
+
+int check_group_ptrs(int n_layers, const flexq_layer_t* layers) {
+  for (int l = 0; l < n_layers; ++l) {
+    const void* ptrs[] = {layers[l].Wq_packed, layers[l].W_scales, layers[l].Y_fp16};
+    const char* names[] = {"layers[].Wq_packed", "layers[].W_scales", "layers[].Y_fp16"};
+    int rc = check_ptrs(3, ptrs, names);
+    if (rc) return rc;
+  }
+  return FLEXQ_OK;
+}
+
+// The grouped launch itself (plan.T <= 64): X is int8 codes with their
+// scales, or (fused) the FP16 activations quantized inside the kernel.
+int launch_group(DeviceState* st, const GroupPlan& g, int M, int K, int gs, int bits, const void* X,
+                 const void* Xs, bool fused, const flexq_layer_t* layers, void* workspace,
+                 cudaStream_t stream) {
+  flexq::LayerTable tab;
+  memset(&tab, 0, sizeof(tab));
+  tab.n_layers = g.n;
+  long long unit = 0, tile0 = 0, part0 = 0;
+  for (int l = 0; l < g.n; ++l) {
+    int rc = encode_scale_map(&tab.sw[l], layers[l].W_scales, layers[l].N, layers[l].N, K / gs, 128);
+    if (rc) return rc;
+    tab.wp[l] = static_cast<const uint8_t*>(layers[l].Wq_packed);
+    tab.y[l] = static_cast<__half*>(layers[l].Y_fp16);
+    tab.N[l] = layers[l].N;
+    tab.unit0[l] = static_cast<int>(unit);
+    tab.n_full[l] = static_cast<int>(g.tiles[l] - g.n_split[l]);
+    tab.split[l] = g.split;
+    tab.tile0[l] = static_cast<int>(tile0);
+    tab.part0[l] = part0;
+    unit += (g.tiles[l] - g.n_split[l]) + g.n_split[l] * g.split;
+    tile0 += g.n_split[l];
+    part0 += g.n_split[l] * g.split * g.T * 128;
+  }
+  tab.unit0[g.n] = static_cast<int>(unit);
+  CUtensorMap map_x, map_sa;
+  memset(&map_x, 0, sizeof(map_x));
+  memset(&map_sa, 0, sizeof(map_sa));
+  int rc = FLEXQ_OK;
+  if (!fused) {
+    if ((rc = encode_x_map(&map_x, X, M, K, g.T))) return rc;
+    if ((rc = encode_scale_map(&map_sa, Xs, M, act_scales_ld(M), K / gs, g.T))) return rc;
+  }
+  flexq::GemmArgs a = {};
+  a.x = fused ? static_cast<const __half*>(X) : nullptr;
+  a.qmax = bits == 6 ? 31 : 127;
+  if (g.split > 1) {
+    a.ws_cnt = static_cast<unsigned int*>(workspace);
+    a.ws_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kCounterBytes);
+  }
+  a.status = st->status;
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  a.M = M; a.K = K; a.gs = gs;
+  a.stall = g_inject_stall.exchange(0);
+  if (fused) return launch_gemm_t<16, false, true>(st, map_x, map_sa, tab, a, g.ctas, stream);
+  switch (g.T) {
+    case 16: return launch_gemm_t<16, false>(st, map_x, map_sa, tab, a, g.ctas, stream);
+    case 32: return launch_gemm_t<32, false>(st, map_x, map_sa, tab, a, g.ctas, stream);
+    default: return launch_gemm_t<64, false>(st, map_x, map_sa, tab, a, g.ctas, stream);
+  }
+}
+
+// Workspace of a grouped GEMM: the grouped plan's split-K region, or for
+// 128-token tiles the largest single layer's (they run one after another).
+size_t group_gemm_bytes(int M, const int* N, int n, int K, int gs, int sms, GroupPlan* out) {
+  GroupPlan g = make_group_plan(M, N, n, K, gs, sms);
+  if (out) *out = g;
+  if (g.T <= 64) return g.ws_bytes;
+  size_t need = 0;
+  for (int l = 0; l < n; ++l)
+    need = std::max(need, workspace_bytes_for(make_plan(M, N[l], K, gs, sms, false), M, N[l]));
+  return need;
+}
+
+int gemm_group_common(int M, int K, int gs, int bits, const int8_t* Xq, const void* Xs,
+                      int n_layers, const flexq_layer_t* layers, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  int N[flexq::kMaxLayers];
+  int rc = check_group(M, K, gs, bits, n_layers, layers, N);
+  if (rc) return rc;
+  if (M == 0) return ok();
+  const void* ptrs[] = {Xq, Xs};
+  const char* names[] = {"Xq", "X_scales"};
+  if ((rc = check_ptrs(2, ptrs, names)) || (rc = check_group_ptrs(n_layers, layers))) return rc;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  GroupPlan g;
+  const size_t need = group_gemm_bytes(M, N, n_layers, K, gs, st->sms, &g);
+  if (g.T > 64) {
+    for (int l = 0; l < n_layers; ++l) {
+      rc = gemm_common(M, layers[l].N, K, gs, Xq, Xs, layers[l].Wq_packed, layers[l].W_scales,
+                       layers[l].Y_fp16, nullptr, false, workspace, workspace_bytes, stream);
+      if (rc) return rc;
+    }
+    return ok();
+  }
+  if (need > 0) {
+    if (workspace == nullptr && workspace_bytes == 0) {
+      g = make_group_plan(M, N, n_layers, K, gs, st->sms, false);   // no workspace: no K split
+    } else if (workspace == nullptr || workspace_bytes < need) {
+      return fail(FLEXQ_ERR_INVALID_ARG, "workspace of %zu bytes at %p, the grouped plan needs %zu",
+                  workspace_bytes, workspace, need);
+    } else if (!aligned16(workspace)) {
+      return fail(FLEXQ_ERR_MISALIGNED, "workspace is not 16-byte aligned");
+    }
+  }
+  rc = launch_group(st, g, M, K, gs, bits, Xq, Xs, false, layers, workspace,
+                    static_cast<cudaStream_t>(stream));
+  return rc ? rc : ok();
+}
+
+// A grouped linear call quantizes inside the GEMM under the same rule as a
+// single layer (16-token tiles, few stages of K per CTA, few tokens); else
+// the activation quantizer writes codes and scales after the GEMM's region
+// of the workspace and the grouped GEMM reads them.
+struct GroupLinearLayout {
+  bool fused;
+  GroupPlan plan;
+  size_t gemm_bytes, xq_off, xs_off, total;
+};
+
+GroupLinearLayout group_linear_layout(int M, const int* N, int n, int K, int gs, int sms) {
+  GroupLinearLayout L = {};
+  L.gemm_bytes = group_gemm_bytes(M, N, n, K, gs, sms, &L.plan);
+  const int route = g_force_linear_route.load();
+  const int stages = (K / 256 + L.plan.split - 1) / L.plan.split;
+  L.fused = L.plan.T == 16 &&
+            (route != 0 ? route == 1 : ((M <= 4 && stages <= 4) || (M <= 8 && stages <= 2)));
+  if (L.fused) {
+    L.total = L.gemm_bytes;
+    return L;
+  }
+  const size_t head = std::max(L.gemm_bytes, kCounterBytes);
+  L.xq_off = (head + 255) & ~static_cast<size_t>(255);
+  L.xs_off = (L.xq_off + static_cast<size_t>(M) * K + 255) & ~static_cast<size_t>(255);
+  L.total = L.xs_off + static_cast<size_t>(K / gs) * act_scales_ld(M) * sizeof(__half);
+  return L;
+}
+
+int linear_group_common(int M, int K, int gs, int bits, const void* X, int n_layers,
+                        const flexq_layer_t* layers, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  int N[flexq::kMaxLayers];
+  int rc = check_group(M, K, gs, bits, n_layers, layers, N);
+  if (rc) return rc;
+  if (M == 0) return ok();
+  const void* ptrs[] = {X};
+  const char* names[] = {"X_fp16"};
+  if ((rc = check_ptrs(1, ptrs, names)) || (rc = check_group_ptrs(n_layers, layers))) return rc;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  const GroupLinearLayout L = group_linear_layout(M, N, n_layers, K, gs, st->sms);
+  if (workspace == nullptr || workspace_bytes < L.total) {
+    if (!(L.total == 0 && workspace == nullptr))
+      return fail(FLEXQ_ERR_INVALID_ARG, "workspace of %zu bytes at %p, the grouped layer needs %zu",
+                  workspace_bytes, workspace, L.total);
+  }
+  if (workspace && !aligned16(workspace)) return fail(FLEXQ_ERR_MISALIGNED, "workspace is not 16-byte aligned");
+  if (L.fused) {
+    rc = launch_group(st, L.plan, M, K, gs, bits, X, nullptr, true, layers, workspace,
+                      static_cast<cudaStream_t>(stream));
+    return rc ? rc : ok();
+  }
+  int8_t* xq = reinterpret_cast<int8_t*>(static_cast<char*>(workspace) + L.xq_off);
+  void* xs = static_cast<char*>(workspace) + L.xs_off;
+  if ((rc = flexq_quantize_act(M, K, gs, bits, X, xq, xs, stream))) return rc;
+  return gemm_group_common(M, K, gs, bits, xq, xs, n_layers, layers, workspace, L.xq_off, stream);
 }
 
 // --------------------------------------------------- static GEMM scratch --
@@ -855,6 +1104,52 @@ int flexq_get_device_status(void* stream) {
                                 "epilogue (scales)"};
   return fail(static_cast<int>(h[0]), "device wait timed out in the %s role of block %u",
               h[1] < 6 ? roles[h[1]] : "?", h[2]);
+}
+
+size_t flexq_gemm_group_workspace_bytes(int M, int K, int group_size, int n_layers,
+                                        const int* N) {
+  if (M <= 0 || K <= 0 || n_layers < 1 || n_layers > flexq::kMaxLayers || !N) return 0;
+  for (int l = 0; l < n_layers; ++l)
+    if (N[l] <= 0 || N[l] % 128 || K % 256 || !valid_gs(group_size) || K % group_size) return 0;
+  return group_gemm_bytes(M, N, n_layers, K, group_size, sm_count_or_default(), nullptr);
+}
+
+size_t flexq_linear_group_workspace_bytes(int M, int K, int group_size, int n_layers,
+                                          const int* N) {
+  if (M <= 0 || K <= 0 || n_layers < 1 || n_layers > flexq::kMaxLayers || !N) return 0;
+  for (int l = 0; l < n_layers; ++l)
+    if (N[l] <= 0 || N[l] % 128 || K % 256 || !valid_gs(group_size) || K % group_size) return 0;
+  return group_linear_layout(M, N, n_layers, K, group_size, sm_count_or_default()).total;
+}
+
+int flexq_group_plan(int M, int K, int group_size, int n_layers, const int* N, int* tile_tokens,
+                     int* k_split, int* ctas, int* launches) {
+  if (M <= 0 || K <= 0 || n_layers < 1 || n_layers > flexq::kMaxLayers || !N)
+    return fail(FLEXQ_ERR_INVALID_ARG, "M=%d K=%d n_layers=%d", M, K, n_layers);
+  for (int l = 0; l < n_layers; ++l) {
+    int rc = check_gemm_shape(M, N[l], K, group_size);
+    if (rc) return rc;
+  }
+  const GroupLinearLayout L = group_linear_layout(M, N, n_layers, K, group_size, sm_count_or_default());
+  if (tile_tokens) *tile_tokens = L.plan.T;
+  if (k_split) *k_split = L.plan.T <= 64 ? L.plan.split : 0;
+  if (ctas) *ctas = L.plan.T <= 64 ? static_cast<int>(L.plan.ctas) : 0;
+  if (launches) *launches = L.fused ? 1 : 1 + (L.plan.T <= 64 ? 1 : n_layers);
+  return ok();
+}
+
+int flexq_gemm_group(int M, int K, int group_size, int act_bits, const int8_t* Xq,
+                     const void* X_scales, int n_layers, const flexq_layer_t* layers,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  return gemm_group_common(M, K, group_size, act_bits, Xq, X_scales, n_layers, layers, workspace,
+                           workspace_bytes, stream);
+}
+
+int flexq_linear_group(int M, int K, int group_size, int act_bits, const void* X_fp16,
+                       int n_layers, const flexq_layer_t* layers, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return linear_group_common(M, K, group_size, act_bits, X_fp16, n_layers, layers, workspace,
+                             workspace_bytes, stream);
 }
 
 #ifdef FLEXQ_TRACE

@@ -75,6 +75,24 @@ struct GemmArgs {
   int stall;               // test hook: withhold the first stage
 };
 
+// The layers of one launch of gemm_w6ax_kernel: one, or up to kMaxLayers
+// layers that read the same activations (a grouped launch: the q, k and v
+// projections, or gate and up), each with its own packed weights, scales,
+// output and K-split plan.  Work units are numbered layer after layer.
+constexpr int kMaxLayers = 4;
+struct LayerTable {
+  CUtensorMap sw[kMaxLayers];      // weight scales [G][N_l], box 128 rows x 8 groups
+  const uint8_t* wp[kMaxLayers];   // packed weights, device form
+  __half* y[kMaxLayers];           // [M, N_l] FP16 outputs
+  long long part0[kMaxLayers];     // first float of the layer's split-K partial tiles
+  int N[kMaxLayers];
+  int unit0[kMaxLayers + 1];       // first work unit of each layer; unit0[n] = all units
+  int n_full[kMaxLayers];          // output tiles run whole (the rest split `split` ways)
+  int split[kMaxLayers];
+  int tile0[kMaxLayers];           // first split-K arrival counter of each layer
+  int n_layers;
+};
+
 template <int T>
 struct GemmCfg {
   // each epilogue warp owns one TMEM lane quarter (32 weight rows) and kCols
@@ -340,7 +358,7 @@ template <int T, bool PARTIALS, bool FUSEDQ = false>
 __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     gemm_w6ax_kernel(const __grid_constant__ CUtensorMap tmap_x,
                      const __grid_constant__ CUtensorMap tmap_sa,
-                     const __grid_constant__ CUtensorMap tmap_sw, const GemmArgs args) {
+                     const __grid_constant__ LayerTable tab, const GemmArgs args) {
   using Cfg = GemmCfg<T>;
   constexpr int STAGES = Cfg::kStages;
   constexpr int ASLOTS = Cfg::kASlots;
@@ -369,21 +387,30 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   // tiles; after them every tile takes `split` consecutive units, one per K
   // range (the plan splits only what would otherwise run as a partial last
   // wave, or everything when there are fewer tiles than SMs)
-  const int unit = blockIdx.x;
+  // the unit's layer, then its output tile and K range within the layer
+  int layer = 0;
+  while (layer + 1 < tab.n_layers && static_cast<int>(blockIdx.x) >= tab.unit0[layer + 1]) ++layer;
+  const int unit = blockIdx.x - tab.unit0[layer];
+  const int n_full = tab.n_full[layer];
   int tile, ks, S;
-  if (unit < args.n_full) {
+  if (unit < n_full) {
     tile = unit;
     ks = 0;
     S = 1;
   } else {
-    const int u = unit - args.n_full;
-    tile = args.n_full + u / args.split;
-    ks = u - (u / args.split) * args.split;
-    S = args.split;
+    const int split = tab.split[layer];
+    const int u = unit - n_full;
+    tile = n_full + u / split;
+    ks = u - (u / split) * split;
+    S = split;
   }
-  const int nt = tile % args.tiles_n;   // weight tile (fastest: neighbours share the tokens)
-  const int mt = tile / args.tiles_n;   // token tile
-  const int M = args.M, N = args.N, K = args.K, gs = args.gs;
+  const int N = tab.N[layer];
+  const int tiles_n = N / kTileRows;
+  const uint8_t* __restrict__ wp = tab.wp[layer];
+  const CUtensorMap* tmap_sw = &tab.sw[layer];
+  const int nt = tile % tiles_n;        // weight tile (fastest: neighbours share the tokens)
+  const int mt = tile / tiles_n;        // token tile
+  const int M = args.M, K = args.K, gs = args.gs;
   const int KB = K / kKBlock;                         // 128-wide weight tiles
   const int units = K / Cfg::kKStage;                 // stages along K (gs | 256)
   const int u0 = static_cast<int>((static_cast<long long>(ks) * units) / S);
@@ -423,7 +450,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     if (!FUSEDQ) prefetch_tensormap(&tmap_x);
     if (!PARTIALS) {
       if (!FUSEDQ) prefetch_tensormap(&tmap_sa);
-      prefetch_tensormap(&tmap_sw);
+      prefetch_tensormap(tmap_sw);
     }
   }
   if (FUSEDQ) {
@@ -464,7 +491,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         if (args.stall && i == 0) continue;
         mbar_arrive_expect_tx(&ctrl->full[i], kStageTx);
         bulk_load(w_ring + i * Cfg::kWStageBytes,
-                  args.wp + (static_cast<size_t>(nt) * KB + kb0 + 2 * i) * kWTileBytes,
+                  wp + (static_cast<size_t>(nt) * KB + kb0 + 2 * i) * kWTileBytes,
                   Cfg::kWStageBytes, &ctrl->full[i]);
       }
       grid_wait_dependencies();
@@ -481,7 +508,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
           uint8_t* dst = sc_ring + slot * Cfg::kScSlotBytes;
           mbar_arrive_expect_tx(&ctrl->s_full[slot], kScTx);
           if (!FUSEDQ) tma_load_2d(dst, &tmap_sa, &ctrl->s_full[slot], mt * T, g0 + 8 * o);
-          tma_load_2d(dst + Cfg::kScSaBytes, &tmap_sw, &ctrl->s_full[slot], nt * kTileRows,
+          tma_load_2d(dst + Cfg::kScSaBytes, tmap_sw, &ctrl->s_full[slot], nt * kTileRows,
                       g0 + 8 * o);
           sc_issued |= 1u << slot;
           sc_parity = (sc_parity & ~(1u << slot)) |
@@ -502,7 +529,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
           mbar_arrive_expect_tx(&ctrl->full[s], kStageTx);
           // tiles (nt, kb) and (nt, kb + 1) are adjacent in the device form
           bulk_load(w_ring + s * Cfg::kWStageBytes,
-                    args.wp + (static_cast<size_t>(nt) * KB + kb) * kWTileBytes,
+                    wp + (static_cast<size_t>(nt) * KB + kb) * kWTileBytes,
                     Cfg::kWStageBytes, &ctrl->full[s]);
         }
         if (!FUSEDQ) {
@@ -831,8 +858,9 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     // last CTA of the output tile to arrive adds the `split` partials in
     // split order (the same order whichever CTA arrives last, so the result
     // is deterministic), writes the FP16 output and resets the counter.
-    const size_t st_idx = static_cast<size_t>(tile - args.n_full);     // split tile index
-    float* part = args.ws_part + st_idx * static_cast<size_t>(S) * T * kTileRows;
+    const size_t st_idx = static_cast<size_t>(tab.tile0[layer] + tile - n_full);   // counter
+    float* part = args.ws_part + tab.part0[layer] +
+                  static_cast<size_t>(tile - n_full) * S * T * kTileRows;
     if (is_epi) {
 #pragma unroll
       for (int j = 0; j < Cfg::kCols; ++j)
@@ -885,7 +913,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     for (int j = 0; j < Cfg::kCols; ++j) {
       const int m = mt * T + col0 + j;
       if (m < M)
-        args.y[static_cast<size_t>(m) * N + n] =
+        tab.y[layer][static_cast<size_t>(m) * N + n] =
             __float2half_rn((j & 1) ? acc[j / 2].y : acc[j / 2].x);
     }
   }

@@ -13,17 +13,19 @@
 //
 // At 128 x 128 outputs per group of 128 codes the per-group rescale is as
 // much work for the CUDA cores as the MMA is for the tensor core, so the
-// layout below is built around the epilogue's instruction count:
-//   * every int32 partial buffer is pre-filled with the bit pattern of the
-//     float 1.5 * 2^23 and the group's MMAs all accumulate onto it, so the
-//     buffer ends holding 1.5 * 2^23 + P' (P' = 4 P, |P'| <= 2^22) as an
-//     exact FP32 value: one packed subtraction (FADD2) per two outputs turns
-//     it into P' with no int -> float conversion;
+// layout below is built around the epilogue:
 //   * the group scales are converted once per CTA into FP32 tables (sa / 4:
 //     the factor 4 of the int8 weight codes folded in), read with 128-bit
 //     broadcast loads;
 //   * eight epilogue warps of 64 tokens each, tensor-memory loads issued one
-//     32-column chunk ahead of the arithmetic.
+//     32-column chunk ahead of the arithmetic, each partial converted with
+//     one int -> float conversion (an exact one: |P| < 2^24) and rescaled
+//     with packed FP32 multiplies and FMAs.
+// (Measured alternatives, all slower at group 128: partial buffers pre-filled
+// with the bits of 1.5 * 2^23 so that a packed subtraction replaces the
+// conversion -- the refill stores cost more than the conversions save; the
+// 16x256b load layout with per-thread scale pairs; sixteen 32-token epilogue
+// warps; a 7-deep ring of 128-code stages.)
 //
 // Warpgroup 0  warp 0  producer: per stage of 256 codes, two TMA boxes of the
 //                      int8 activations (128 rows x 128 B, 128-byte swizzle)
@@ -87,31 +89,28 @@ struct WideCtrl {
   uint32_t is_last;        // split-K: this CTA reduces the output tile
 };
 
-// 1.5 * 2^23: a float whose unit in the last place is 1, so its bit pattern
-// plus an integer p with |p| <= 2^22 is the bit pattern of 1.5 * 2^23 + p
-constexpr uint32_t kPartialBias = 0x4B400000u;
-constexpr float kPartialBiasF = 12582912.0f;
-
-// The partial's 32 columns of one chunk, minus the bias, into the FP32
-// accumulators: acc[j] += P'[j] * sa4[j] * sw (sa4 = sa / 4 from the table).
+// The partial's 32 columns of one chunk into the FP32 accumulators:
+// acc[j] += P'[j] * sa4[j] * sw (P' = 4 P from the code * 4 weights, sa4 =
+// sa / 4 from the table); |P'| <= 2^22, so the conversion is exact.
 __device__ __forceinline__ void wide_rescale_chunk(const uint32_t (&pv)[32], const float* sa,
                                                    float sw, float2* acc) {
   const float2 sw2 = make_float2(sw, sw);
-  const float2 nb = make_float2(-kPartialBiasF, -kPartialBiasF);
   const float4* sa4 = reinterpret_cast<const float4*>(sa);
 #pragma unroll
   for (int j = 0; j < 32; j += 4) {
     const float4 s4 = sa4[j / 4];
     const float2 s_lo = __fmul2_rn(sw2, make_float2(s4.x, s4.y));
     const float2 s_hi = __fmul2_rn(sw2, make_float2(s4.z, s4.w));
-    const float2 p_lo = __fadd2_rn(make_float2(__uint_as_float(pv[j]), __uint_as_float(pv[j + 1])), nb);
-    const float2 p_hi = __fadd2_rn(make_float2(__uint_as_float(pv[j + 2]), __uint_as_float(pv[j + 3])), nb);
+    const float2 p_lo = make_float2(__int2float_rn(static_cast<int32_t>(pv[j])),
+                                    __int2float_rn(static_cast<int32_t>(pv[j + 1])));
+    const float2 p_hi = make_float2(__int2float_rn(static_cast<int32_t>(pv[j + 2])),
+                                    __int2float_rn(static_cast<int32_t>(pv[j + 3])));
     acc[j / 2] = __ffma2_rn(p_lo, s_lo, acc[j / 2]);
     acc[j / 2 + 1] = __ffma2_rn(p_hi, s_hi, acc[j / 2 + 1]);
   }
 }
 
-// Debug export: the chunk's exact int32 partials P = (bits - bias) / 4.
+// Debug export: the chunk's exact int32 partials P = P' / 4.
 __device__ __forceinline__ void wide_store_partials(const uint32_t (&pv)[32], int32_t* p, int g,
                                                     int M, int N, int m0, int n) {
 #pragma unroll
@@ -119,7 +118,7 @@ __device__ __forceinline__ void wide_store_partials(const uint32_t (&pv)[32], in
     const int m = m0 + j;
     if (m < M)
       p[(static_cast<size_t>(g) * M + m) * N + n] =
-          static_cast<int32_t>(pv[j] - kPartialBias) >> 2;
+          static_cast<int32_t>(pv[j]) >> 2;
   }
 }
 
@@ -275,8 +274,8 @@ __global__ void __launch_bounds__(WideCfg::kThreads, 1)
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA ----
       // The MMAs of a group form one straight run (the group size is a
-      // compile-time constant); the waits sit before a group's first MMA.
-      // Every MMA accumulates (the buffers start at the bias).
+      // compile-time constant); the waits sit before a group's first MMA,
+      // whose first K slice starts a fresh accumulator.
       if (lane == 0) {
         const uint64_t desc0 = smem_desc_k_sw128(smem_u32(xs_ring));
         auto run = [&](auto gs_c) -> bool {
@@ -294,7 +293,7 @@ __global__ void __launch_bounds__(WideCfg::kThreads, 1)
 #pragma unroll
             for (int j = 0; j < G; ++j) {
               // use u of a buffer follows phase u of its release barrier
-              // (phase 0: the epilogue's first fill)
+              // (phase 0: the epilogue's start)
               if (!mbar_wait(&ctrl->p_empty[pb.idx], pb.phase, lim)) return false;
               tc_fence_after();
               const uint32_t d_col = tmem + Cfg::kPCol0 + pb.idx * T;
@@ -303,7 +302,7 @@ __global__ void __launch_bounds__(WideCfg::kThreads, 1)
                 const int sub = j * SPG + k;
                 mma_i8_tmem_a(d_col, a_col + sub * 8,
                               b_desc + (((sub >> 2) * Cfg::kXsHalf + (sub & 3) * 32) >> 4), idesc,
-                              1u);
+                              k == 0 ? 0u : 1u);
               }
               mma_commit(&ctrl->p_full[pb.idx]);
               pb.next();
@@ -431,14 +430,7 @@ __global__ void __launch_bounds__(WideCfg::kThreads, 1)
     auto pcol = [&](int b, int c) -> uint32_t {
       return tmem + lane_base + Cfg::kPCol0 + b * T + col_h + 32 * c;
     };
-    // phase 0 of every release barrier: the buffers hold the bias
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      tmem_fill32(pcol(b, 0), kPartialBias);
-      tmem_fill32(pcol(b, 1), kPartialBias);
-    }
-    tmem_wait_st();
-    tc_fence_before();
+    // phase 0 of every release barrier: every buffer is free at the start
     __syncwarp();
     if (lane == 0)
       for (int b = 0; b < NB; ++b) mbar_arrive(&ctrl->p_empty[b]);
@@ -466,18 +458,15 @@ __global__ void __launch_bounds__(WideCfg::kThreads, 1)
       const float* sa_g = tab + gi * 128 + col_h;
       const float sw = PARTIALS ? 0.0f : tab[Cfg::kScFloats + gi * 128 + row];
       const int b = pb.idx;
-      // chunk 0 has landed (issued one chunk ago); request chunk 1, refill
-      // chunk 0 with the bias, then rescale chunk 0 while chunk 1 loads
+      // chunk 0 has landed (issued one chunk ago); request chunk 1, then
+      // rescale chunk 0 while chunk 1 loads
       tmem_wait_ld();
       tmem_ld32(pcol(b, 1), pc);
-      tmem_fill32(pcol(b, 0), kPartialBias);
       if (PARTIALS)
         wide_store_partials(pa, args.p, g, M, N, mt * T + col_h, n);
       else
         wide_rescale_chunk(pa, sa_g, sw, acc);
       tmem_wait_ld();
-      tmem_fill32(pcol(b, 1), kPartialBias);
-      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->p_empty[b]);

@@ -22,6 +22,13 @@ FLEXQ_ERR_CUDA = 4
 FLEXQ_ERR_DEVICE_TIMEOUT = 5
 
 _lib = None
+MAX_GROUP_LAYERS = 4
+
+
+class Layer(ctypes.Structure):
+    """flexq_layer_t: one layer of a grouped call."""
+    _fields_ = [("N", ctypes.c_int), ("Wq_packed", ctypes.c_void_p),
+                ("W_scales", ctypes.c_void_p), ("Y_fp16", ctypes.c_void_p)]
 
 
 class FlexQError(RuntimeError):
@@ -77,6 +84,18 @@ def lib():
             "flexq_set_wait_limit_ns": (c_int, [ctypes.c_uint64]),
             "flexq_debug_inject_stall": (c_int, [c_int]),
             "flexq_get_device_status": (c_int, [c_void_p]),
+            "flexq_gemm_group": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_int,
+                                         ctypes.POINTER(Layer), c_void_p, c_size_t, c_void_p]),
+            "flexq_linear_group": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_int,
+                                           ctypes.POINTER(Layer), c_void_p, c_size_t,
+                                           c_void_p]),
+            "flexq_gemm_group_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int,
+                                                            ctypes.POINTER(c_int)]),
+            "flexq_linear_group_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int,
+                                                              ctypes.POINTER(c_int)]),
+            "flexq_group_plan": (c_int, [c_int, c_int, c_int, c_int, ctypes.POINTER(c_int),
+                                         ctypes.POINTER(c_int), ctypes.POINTER(c_int),
+                                         ctypes.POINTER(c_int), ctypes.POINTER(c_int)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -339,3 +358,78 @@ def device_status(device=None):
     if st == FLEXQ_ERR_DEVICE_TIMEOUT:
         reset_workspaces()
     return st, msg
+
+
+# ------------------------------------------------------------ grouped calls
+def _n_array(Ns):
+    return (ctypes.c_int * len(Ns))(*Ns)
+
+
+def group_plan(M, K, group_size, Ns):
+    """(tokens per tile, K split, CTAs, launches of linear_group) for layers of
+    widths Ns that share their activations."""
+    t, s, c, n = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(lib().flexq_group_plan(M, K, group_size, len(Ns), _n_array(Ns), ctypes.byref(t),
+                                  ctypes.byref(s), ctypes.byref(c), ctypes.byref(n)))
+    return t.value, s.value, c.value, n.value
+
+
+def gemm_group_workspace_bytes(M, K, group_size, Ns):
+    return int(lib().flexq_gemm_group_workspace_bytes(M, K, group_size, len(Ns), _n_array(Ns)))
+
+
+def linear_group_workspace_bytes(M, K, group_size, Ns):
+    return int(lib().flexq_linear_group_workspace_bytes(M, K, group_size, len(Ns), _n_array(Ns)))
+
+
+def _layers(weights, outs, K, group_size, M, device):
+    if not 1 <= len(weights) <= MAX_GROUP_LAYERS:
+        raise ValueError(f"1..{MAX_GROUP_LAYERS} layers, got {len(weights)}")
+    arr = (Layer * len(weights))()
+    ys = []
+    for i, (wp, ws, N) in enumerate(weights):
+        _need(wp, "wp", torch.uint8, (weight_packed_bytes(N, K, group_size),))
+        _need(ws, "ws", torch.float16, (K // group_size, N))
+        y = outs[i] if outs is not None and outs[i] is not None else \
+            torch.empty(M, N, dtype=torch.float16, device=device)
+        _need(y, "out", torch.float16, (M, N))
+        arr[i] = Layer(N, wp.data_ptr(), ws.data_ptr(), y.data_ptr())
+        ys.append(y)
+    return arr, ys
+
+
+def _ws_args(buf, device, need):
+    if buf is None:
+        buf = workspace(device, need) if need else None
+    if buf is None or buf.numel() == 0:
+        return ctypes.c_void_p(0), 0
+    _need(buf, "workspace", torch.uint8)
+    return _ptr(buf), buf.numel()
+
+
+def gemm_group(xq, xs, weights, group_size, act_bits=6, outs=None, workspace_buf=None):
+    """One launch of the group GEMM for layers sharing quantized activations:
+    weights = [(wp, ws, N), ...] (1..4 layers); returns their FP16 outputs."""
+    _need(xq, "xq", torch.int8)
+    M, K = xq.shape
+    _need(xs, "xs", torch.float16, (K // group_size, act_scales_ld(M)))
+    arr, ys = _layers(weights, outs, K, group_size, M, xq.device)
+    wsp, wsn = _ws_args(workspace_buf, xq.device,
+                        gemm_group_workspace_bytes(M, K, group_size, [w[2] for w in weights]))
+    _check(lib().flexq_gemm_group(M, K, group_size, act_bits, _ptr(xq), _ptr(xs), len(weights),
+                                  arr, wsp, wsn, _stream(xq)))
+    return ys
+
+
+def linear_group(x, weights, group_size, act_bits=6, outs=None, workspace_buf=None):
+    """Layers [(wp, ws, N), ...] that read the same FP16 activations x [M, K],
+    quantized once (act_bits 6 or 8), in one grouped launch (or the
+    quantizer and one grouped launch); returns their FP16 outputs."""
+    _need(x, "x", torch.float16)
+    M, K = x.shape
+    arr, ys = _layers(weights, outs, K, group_size, M, x.device)
+    wsp, wsn = _ws_args(workspace_buf, x.device,
+                        linear_group_workspace_bytes(M, K, group_size, [w[2] for w in weights]))
+    _check(lib().flexq_linear_group(M, K, group_size, act_bits, _ptr(x), len(weights), arr, wsp,
+                                    wsn, _stream(x)))
+    return ys

@@ -14,7 +14,12 @@ GEMM (flexq.linear_launches == 1), flexq.linear; otherwise the site is
 quantized once (flexq.quantize_act) for this and later layers.  Every output
 is bit-identical to flexq.linear on that layer alone.
 
-With fuse_sites=True the layers of one site and width are also merged into
+With group_sites=True (the default) the layers of one site and width run as
+one grouped call (flexq.linear_group): one quantization and one kernel
+launch for, e.g., q, k and v, each layer keeping its own packed weights and
+output.
+
+With fuse_sites=True the layers of one site and width are instead merged into
 one GEMM (the fused q/k/v and gate/up projections of inference engines):
 their FP16 weights are stacked along N and quantized as one matrix (the
 quantization is per row, so every layer keeps its codes and scales), and
@@ -81,15 +86,18 @@ class LayerStack:
     config:     see the module docstring;
     weights:    {name: FP16 [N, K] tensor} (any device), or None for seeded
                 synthetic weights drawn on `device` (N(0, std));
-    fuse_sites: merge the layers of one site and width into one GEMM.
+    fuse_sites: merge the layers of one site and width into one GEMM;
+    group_sites: run the layers of one site and width as one grouped call
+                 (ignored with fuse_sites).
     """
 
     def __init__(self, layers, config, device="cuda", weights=None, std=0.015, seed=0,
-                 fuse_sites=False):
+                 fuse_sites=False, group_sites=True):
         self.layers = list(layers)
         self.gs, self.bits = parse_config(config, self.layers)
         self.device = torch.device(device)
         self.fuse_sites = fuse_sites
+        self.group_sites = group_sites and not fuse_sites
         self.site_k = {}
         for name, N, K, site in self.layers:
             if self.site_k.setdefault(site, K) != K:
@@ -121,6 +129,16 @@ class LayerStack:
                 w = torch.cat([weight(name, N, K) for name, N, _ in members], dim=0)
             self.packed[key] = flexq.quantize_weight(w, self.gs)
             del w
+        # grouped calls: the units of one (site, bits), in order of first use
+        self.groups = []
+        by_q = {}
+        for i, (key, site, bits, K, members, n_total) in enumerate(self.units):
+            q = (site, bits)
+            if self.group_sites and q in by_q:
+                self.groups[by_q[q]].append(i)
+            else:
+                by_q[q] = len(self.groups)
+                self.groups.append([i])
         self._ybuf = {}
 
     def sites(self):
@@ -141,6 +159,12 @@ class LayerStack:
 
     def launches(self, M):
         """Kernel launches of one forward at batch M."""
+        if self.group_sites:
+            n = 0
+            for g in self.groups:
+                K = self.units[g[0]][3]
+                n += flexq.group_plan(M, K, self.gs, [self.units[i][5] for i in g])[3]
+            return n
         n, quantized = 0, set()
         for key, site, bits, K, members, n_total in self.units:
             q = (site, bits)
@@ -166,6 +190,15 @@ class LayerStack:
             elif x.shape[0] != M:
                 raise ValueError("every site must hold the same number of tokens")
         out = {} if out is None else out
+        if self.group_sites:
+            for g in self.groups:
+                key, site, bits, K, members, n_total = self.units[g[0]]
+                weights = [self.packed[self.units[i][0]] + (self.units[i][5],) for i in g]
+                outs = [out.get(self.units[i][4][0][0]) for i in g]
+                ys = flexq.linear_group(acts[site], weights, self.gs, bits, outs=outs)
+                for i, y in zip(g, ys):
+                    out[self.units[i][4][0][0]] = y
+            return out
         codes = {}
         for key, site, bits, K, members, n_total in self.units:
             wp, ws = self.packed[key]

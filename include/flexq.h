@@ -251,6 +251,80 @@ int flexq_gemm_static_scratch(int M, int N, int K, int group_size, int act_bits,
                               void* Y_fp16, void* stream);
 
 /*
+ * One layer of a grouped call: layers that read the same activations (the
+ * q, k and v projections of attention, or the gate and up projections of an
+ * MLP), each with its own weights and output.
+ *   N          output channels of this layer (N % 128 == 0);
+ *   Wq_packed  its packed 6-bit weights (device form, flexq_quantize_weight);
+ *   W_scales   its FP16 weight scales, group-major [K/gs, N];
+ *   Y_fp16     its FP16 output [M, N] (written, not read).
+ */
+typedef struct flexq_layer {
+  int N;
+  const void* Wq_packed;
+  const void* W_scales;
+  void* Y_fp16;
+} flexq_layer_t;
+
+#define FLEXQ_MAX_GROUP_LAYERS 4
+
+/*
+ * flexq_gemm_group -- the GEMM of flexq_gemm_w6a6 / w6a8 for 1 to 4 layers
+ * that share their quantized activations (Xq, X_scales as for those calls;
+ * act_bits 6 or 8 only names the code range), in one kernel launch for
+ * batches of at most 64 tokens and one launch per layer above.  The method
+ * is per layer exactly that of flexq_gemm_w6a6/w6a8 (FlexQ arXiv abstract;
+ * drgamma blog, "Bridging Software and Hardware with BTC"); grouping the
+ * layers is this library's launch strategy: one set of CTAs streams every
+ * layer's weights, so that one layer's set-up and split-K tail overlap the
+ * others' streaming.  The plan is shared: the token tile follows M, and when
+ * all layers together have fewer output tiles than CTA slots every tile is
+ * split along K by one factor (split-K partials in the workspace, added in
+ * split order: results are deterministic, and equal to a single-layer call
+ * with the same split).
+ *   workspace  zero-filled device buffer of flexq_gemm_group_workspace_bytes
+ *              bytes (NULL and 0 run without a K split), left zero.
+ * Errors: FLEXQ_ERR_INVALID_ARG for n_layers outside 1..4, a NULL `layers`,
+ * bad act_bits or a short workspace; the shape and pointer rules of
+ * flexq_gemm_w6a6 per layer.
+ */
+int flexq_gemm_group(int M, int K, int group_size, int act_bits, const int8_t* Xq,
+                     const void* X_scales, int n_layers, const flexq_layer_t* layers,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of flexq_gemm_group (0 for invalid arguments). */
+size_t flexq_gemm_group_workspace_bytes(int M, int K, int group_size, int n_layers,
+                                        const int* N);
+
+/*
+ * flexq_linear_group -- flexq_linear_w6a6 / w6a8 (act_bits 6 or 8) for 1 to
+ * 4 layers that read the same FP16 activations X [M, K]: the activations are
+ * quantized once, inside the grouped GEMM launch where a single layer would
+ * be (16-token tiles, few K stages per CTA, a few tokens), else by one
+ * activation-quantizer launch into the workspace, followed by
+ * flexq_gemm_group on those codes.  Every output equals flexq_linear_* on
+ * that layer alone up to the FP32 summation order of the K split.
+ *   workspace  zero-filled device buffer of flexq_linear_group_workspace_bytes
+ *              bytes (may be NULL when that is 0).
+ */
+int flexq_linear_group(int M, int K, int group_size, int act_bits, const void* X_fp16,
+                       int n_layers, const flexq_layer_t* layers, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of flexq_linear_group (0 for invalid arguments). */
+size_t flexq_linear_group_workspace_bytes(int M, int K, int group_size, int n_layers,
+                                          const int* N);
+
+/*
+ * flexq_group_plan -- host only: the grouped plan for these layers: tokens
+ * per tile, K split and CTAs of the grouped launch (0 and 0 when the batch
+ * takes 128-token tiles and the layers run one launch each), and the kernel
+ * launches of flexq_linear_group.
+ */
+int flexq_group_plan(int M, int K, int group_size, int n_layers, const int* N, int* tile_tokens,
+                     int* k_split, int* ctas, int* launches);
+
+/*
  * flexq_debug_check_quantizer -- test hook: runs the GPU quantizer's
  * division-free code rule against the IEEE-division rule (FP32 division by
  * the stored FP16 scale, round half to even, clamp) on every pair of a

@@ -178,3 +178,34 @@ def test_static_scratch_validation_before_any_launch(L):
     assert b"X_scales" in L.flexq_last_error_message()
     assert f(4, 256, 256, 128, 8, FAKE, FAKE, FAKE, FAKE, MISALIGNED, NULL) == \
         flexq.FLEXQ_ERR_MISALIGNED
+
+
+def test_group_validation_before_any_launch(L):
+    Layer = flexq.Layer
+    arr = (Layer * 2)(Layer(256, 1 << 20, 1 << 20, 1 << 20), Layer(384, 1 << 20, 1 << 20, 1 << 20))
+    g = L.flexq_gemm_group
+    assert g(4, 256, 128, 6, FAKE, FAKE, 0, arr, NULL, 0, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert g(4, 256, 128, 6, FAKE, FAKE, 5, arr, NULL, 0, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert g(4, 256, 128, 6, FAKE, FAKE, 2, None, NULL, 0, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert g(4, 256, 128, 7, FAKE, FAKE, 2, arr, NULL, 0, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    bad = (Layer * 1)(Layer(200, 1 << 20, 1 << 20, 1 << 20))
+    assert g(4, 256, 128, 6, FAKE, FAKE, 1, bad, NULL, 0, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
+    assert g(4, 256, 128, 6, NULL, FAKE, 2, arr, NULL, 0, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    nul = (Layer * 1)(Layer(256, 1 << 20, 0, 1 << 20))
+    assert g(4, 256, 128, 6, FAKE, FAKE, 1, nul, NULL, 0, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert g(0, 256, 128, 6, FAKE, FAKE, 2, arr, NULL, 0, NULL) == flexq.FLEXQ_OK
+    f = L.flexq_linear_group
+    assert f(4, 256, 128, 8, NULL, 2, arr, NULL, 0, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert f(4, 256, 48, 8, FAKE, 2, arr, NULL, 0, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED
+
+
+def test_group_plan_is_host_only_and_sane(L):
+    # LLaMA-2-70B q/k/v at one token: 80 weight tiles, split 3 -> 240 CTAs
+    assert flexq.group_plan(1, 8192, 128, [8192, 1024, 1024])[:3] == (16, 3, 240)
+    # one layer: the grouped plan splits like the single-layer one when it fits a wave
+    t, s, c, n = flexq.group_plan(1, 4096, 128, [4096])
+    assert (t, s, c) == flexq.plan(1, 4096, 4096, 128)
+    # 128-token tiles: one launch per layer after the quantizer
+    assert flexq.group_plan(512, 8192, 128, [28672, 28672]) == (128, 0, 0, 3)
+    assert flexq.gemm_group_workspace_bytes(1, 8192, 128, [8192, 1024, 1024]) == \
+        4096 + 80 * 3 * 16 * 128 * 4

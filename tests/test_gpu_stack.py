@@ -1,7 +1,8 @@
-"""The mixed W6A6 / W6A8 layer stack on the GPU: every layer's output is
-bit-identical to flexq.linear on that layer alone (the stack only shares the
-quantization of a site between layers of the same bit width), and within the
-GEMM tolerance of the oracle's linear layer."""
+"""The mixed W6A6 / W6A8 layer stack on the GPU: run layer by layer, every
+layer's output is bit-identical to flexq.linear on that layer alone (the
+stack only shares the quantization of a site between layers of the same bit
+width); run with grouped calls, to flexq.linear_group on the site's layers;
+always within the GEMM tolerance of the oracle's linear layer."""
 
 import pytest
 import torch
@@ -33,7 +34,7 @@ def _acts(layers, M, seed):
 def test_small_block_matches_single_layers_and_the_oracle(M):
     w = {name: inputs.weights(N, K, std=0.015, seed=inputs.layer_seed("stack-w", name))
          for name, N, K, _ in SMALL}
-    st = stack.LayerStack(SMALL, MIXED, weights=w)
+    st = stack.LayerStack(SMALL, MIXED, weights=w, group_sites=False)
     acts = _acts(SMALL, M, seed=M)
     dacts = {k: v.cuda() for k, v in acts.items()}
     out = st.forward(dacts)
@@ -48,7 +49,7 @@ def test_small_block_matches_single_layers_and_the_oracle(M):
 
 @pytest.mark.parametrize("M", [1, 16])
 def test_70b_block_matches_single_layers(M):
-    st = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED)
+    st = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED, group_sites=False)
     acts = {k: v.cuda() for k, v in _acts(inputs.LLAMA2_70B_BLOCK, M, seed=70).items()}
     out = st.forward(acts)
     for name, N, K, site in inputs.LLAMA2_70B_BLOCK:
@@ -59,14 +60,14 @@ def test_70b_block_matches_single_layers(M):
 
 
 def test_launch_count_shares_site_quantization():
-    st = stack.LayerStack(SMALL, MIXED)
+    st = stack.LayerStack(SMALL, MIXED, group_sites=False)
     assert st.launches(1) == 7                       # quantization inside each GEMM
     # M = 40: attn_in has 6-bit q, v and 8-bit k (2 quantizations + 3 GEMMs),
     # attn_out 2, mlp_in 1 + 2, mlp_act 2
     assert st.launches(40) == 5 + 2 + 3 + 2
     # the 70B block at M = 1: q (8 stages per CTA) quantizes attn_in for k and
     # v too; o, gate and down quantize first; up reuses gate's codes
-    big = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED)
+    big = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED, group_sites=False)
     assert big.launches(1) == 2 + 1 + 1 + 2 + 2 + 1 + 2
 
 
@@ -108,6 +109,38 @@ def test_fused_70b_block_launches():
     assert [len(u[4]) for u in st.units] == [3, 1, 2, 1]      # qkv, o, gate+up, down
     assert st.launches(16) == 4 * 2
     acts = {k: v.cuda() for k, v in _acts(inputs.LLAMA2_70B_BLOCK, 16, seed=71).items()}
+    out = st.forward(acts)
+    assert out["k"].shape == (16, 1024) and out["up"].shape == (16, 28672)
+    assert flexq.device_status()[0] == flexq.FLEXQ_OK
+
+
+@pytest.mark.parametrize("M", [1, 5, 40])
+def test_grouped_small_block_matches_grouped_calls_and_the_oracle(M):
+    w = {name: inputs.weights(N, K, std=0.015, seed=inputs.layer_seed("stack-w", name))
+         for name, N, K, _ in SMALL}
+    st = stack.LayerStack(SMALL, MIXED, weights=w)            # grouped by default
+    # attn_in: q, v (6 bits) grouped, k (8 bits) alone; mlp_in: gate + up
+    assert sorted(len(g) for g in st.groups) == [1, 1, 1, 2, 2]
+    acts = _acts(SMALL, M, seed=M + 3)
+    dacts = {k: v.cuda() for k, v in acts.items()}
+    out = st.forward(dacts)
+    for g in st.groups:
+        names = [st.units[i][4][0][0] for i in g]
+        site, bits = st.units[g[0]][1], st.units[g[0]][2]
+        ys = flexq.linear_group(dacts[site], [st.layer_weights(n) for n in names], 128, bits)
+        for n, y in zip(names, ys):
+            assert torch.equal(out[n], y), n
+    for name, N, K, site in SMALL:
+        ref = orc.linear_layer(acts[site].numpy(), w[name].numpy(), 128, MIXED["act_bits"][name])
+        assert_within(np16(out[name]), ref["y64"], TOL)
+
+
+def test_grouped_70b_block_launches_and_runs():
+    st = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED)
+    # q/k/v and gate/up grouped: quantizer + one grouped launch each, o and
+    # down quantizer + GEMM
+    assert st.launches(1) == 2 + 2 + 2 + 2
+    acts = {k: v.cuda() for k, v in _acts(inputs.LLAMA2_70B_BLOCK, 16, seed=72).items()}
     out = st.forward(acts)
     assert out["k"].shape == (16, 1024) and out["up"].shape == (16, 28672)
     assert flexq.device_status()[0] == flexq.FLEXQ_OK
