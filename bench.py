@@ -280,6 +280,17 @@ class Layers:
             wp, ws = flexq.quantize_weight(w16, GS)
             del w16
             self.w.append((name, N, K, bits, site, wp, ws))
+        # layers that read the same input at the same width share one call
+        # (flexq.linear_group / one quantization): gate and up
+        self.groups = []
+        by_q = {}
+        for layer in self.w:
+            q = (layer[4], layer[3])
+            if q in by_q:
+                self.groups[by_q[q]].append(layer)
+            else:
+                by_q[q] = len(self.groups)
+                self.groups.append([layer])
         self.x, self.xq, self.xs, self.y = {}, {}, {}, {}
         sites = {site: K for (_, _, K, _, site) in layers}
         for M in ms:
@@ -307,42 +318,57 @@ class Layers:
         from bit_group_quantized_flexq_b200 import flexq
         n = 0
         for M in self.ms:
-            for (_, N, K, _, _, _, _) in self.w:
-                n += 2 if self.split_m(M) else flexq.linear_launches(M, N, K, GS)
+            for g in self.groups:
+                if self.split_m(M):
+                    n += 1 + len(g)
+                else:
+                    n += flexq.group_plan(M, g[0][2], GS, [l[1] for l in g])[3]
         return n
 
-    def quant(self, M, layer):
+    def quant(self, M, group):
+        """One quantization of the group's input (codes kept under its first layer)."""
         from bit_group_quantized_flexq_b200 import flexq
-        name, _, _, bits, site, _, _ = layer
+        name, _, _, bits, site, _, _ = group[0]
         flexq.quantize_act(self.x[(M, site)], GS, bits,
                            out=(self.xq[(M, name)], self.xs[(M, name)]))
 
-    def gemm(self, M, layer):
+    def gemm(self, M, group, layer):
         from bit_group_quantized_flexq_b200 import flexq
+        first = group[0][0]
         name, N, K, bits, _, wp, ws = layer
-        flexq.gemm(self.xq[(M, name)], self.xs[(M, name)], wp, ws, N, GS, bits,
+        flexq.gemm(self.xq[(M, first)], self.xs[(M, first)], wp, ws, N, GS, bits,
                    out=self.y[(M, name)])
 
-    def linear(self, M, layer):
+    def linear(self, M, group):
+        """The group's layers from FP16 activations: one flexq.linear, or one
+        grouped call (flexq.linear_group) for layers sharing their input."""
         from bit_group_quantized_flexq_b200 import flexq
-        name, N, K, bits, site, wp, ws = layer
-        flexq.linear(self.x[(M, site)], wp, ws, N, GS, bits, out=self.y[(M, name)])
+        if len(group) == 1:
+            name, N, K, bits, site, wp, ws = group[0]
+            flexq.linear(self.x[(M, site)], wp, ws, N, GS, bits, out=self.y[(M, name)])
+            return
+        bits, site = group[0][3], group[0][4]
+        flexq.linear_group(self.x[(M, site)], [(l[5], l[6], l[1]) for l in group], GS, bits,
+                           outs=[self.y[(M, l[0])] for l in group])
 
     def run_m(self, M):
-        for layer in self.w:
-            self.linear(M, layer)
+        for group in self.groups:
+            self.linear(M, group)
 
     def segments(self):
         """The step cut into replayable pieces: at the HBM-bound M all layers
-        of an M are one piece (flexq.linear per layer); at the tensor-bound M
-        every quantization and every GEMM is its own piece so that events can
-        bracket the GEMM launches."""
+        of an M are one piece (flexq.linear per layer, flexq.linear_group for
+        gate and up); at the tensor-bound M every quantization (one per input)
+        and every GEMM is its own piece so that events can bracket the GEMM
+        launches."""
         segs = []
         for M in self.ms:
             if self.split_m(M):
-                for layer in self.w:
-                    segs.append(("quant", M, layer, (lambda M=M, l=layer: self.quant(M, l))))
-                    segs.append(("gemm", M, layer, (lambda M=M, l=layer: self.gemm(M, l))))
+                for group in self.groups:
+                    segs.append(("quant", M, group[0], (lambda M=M, g=group: self.quant(M, g))))
+                    for layer in group:
+                        segs.append(("gemm", M, layer,
+                                     (lambda M=M, g=group, l=layer: self.gemm(M, g, l))))
             else:
                 segs.append(("all", M, None, (lambda M=M: self.run_m(M))))
         return segs
@@ -576,24 +602,25 @@ def gemm_diagnostics(W, device, hbm_gbs, int8_peak_tops, reps=None):
     `reps` rounds of them back to back (the other layers' weights stream in
     between, so each launch reads its weights cold); events bracket the graph
     replay, so host launch work is not timed.  `gemm_*`: the GEMM alone on
-    quantized activations; `linear_*`: the whole layer from FP16 activations
-    through flexq.linear."""
+    quantized activations; `linear_*`: the whole layers from FP16 activations
+    through flexq.linear (flexq.linear_group for gate and up)."""
     import torch
     from bit_group_quantized_flexq_b200 import flexq
     out = []
     stream = torch.cuda.Stream(device)
     for M in W.ms:
-        for layer in W.w:
-            W.quant(M, layer)                     # the GEMM's quantized inputs
+        for group in W.groups:
+            W.quant(M, group)                     # the GEMMs' quantized inputs
         n_reps = reps or (2 if M >= 4096 else 5)
 
         def gemm_body():
-            for layer in W.w:
-                W.gemm(M, layer)
+            for group in W.groups:
+                for layer in group:
+                    W.gemm(M, group, layer)
 
         def linear_body():
-            for layer in W.w:
-                W.linear(M, layer)
+            for group in W.groups:
+                W.linear(M, group)
 
         t_us = _graph_time_us(gemm_body, device, stream, n_reps)
         l_us = _graph_time_us(linear_body, device, stream, n_reps)

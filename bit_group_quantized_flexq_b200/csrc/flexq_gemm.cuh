@@ -447,6 +447,20 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       }
     }
     fence_barrier_init();
+    // The packed weights are read-only inputs: the first ring's worth is
+    // requested at once, before the TMEM allocation and the CTA barrier, and
+    // before waiting for the kernels this one depends on (whose outputs may
+    // be this kernel's activations and their scales).  With fused
+    // quantization a stage's copy is the weights alone.
+    constexpr uint32_t kStageTx0 = FUSEDQ ? Cfg::kWStageBytes : Cfg::kStageBytes;
+    const int n_pre = nst < STAGES ? nst : STAGES;
+    for (int i = 0; i < n_pre; ++i) {
+      if (args.stall && i == 0) continue;
+      mbar_arrive_expect_tx(&ctrl->full[i], kStageTx0);
+      bulk_load(w_ring + i * Cfg::kWStageBytes,
+                wp + (static_cast<size_t>(nt) * KB + kb0 + 2 * i) * kWTileBytes,
+                Cfg::kWStageBytes, &ctrl->full[i]);
+    }
     if (!FUSEDQ) prefetch_tensormap(&tmap_x);
     if (!PARTIALS) {
       if (!FUSEDQ) prefetch_tensormap(&tmap_sa);
@@ -479,21 +493,12 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       const int n_oct = PARTIALS ? 0 : (ngroups + 7) / 8;
       int next_oct = 0;
       bool ok = true;
-      // The packed weights are read-only inputs: the first ring's worth is
-      // requested before waiting for the kernels this one depends on (whose
-      // outputs may be this kernel's activations and their scales).
+      // the first ring's weights were requested during set-up; with fused
+      // quantization the stage's copy is the weights alone, and the scale
+      // slots receive the weight scales only
       const int n_pre = nst < STAGES ? nst : STAGES;
-      // with fused quantization the stage's copy is the weights alone, and
-      // the scale slots receive the weight scales only
       constexpr uint32_t kStageTx = FUSEDQ ? Cfg::kWStageBytes : Cfg::kStageBytes;
       constexpr uint32_t kScTx = FUSEDQ ? Cfg::kScSlotBytes - Cfg::kScSaBytes : Cfg::kScSlotBytes;
-      for (int i = 0; i < n_pre; ++i) {
-        if (args.stall && i == 0) continue;
-        mbar_arrive_expect_tx(&ctrl->full[i], kStageTx);
-        bulk_load(w_ring + i * Cfg::kWStageBytes,
-                  wp + (static_cast<size_t>(nt) * KB + kb0 + 2 * i) * kWTileBytes,
-                  Cfg::kWStageBytes, &ctrl->full[i]);
-      }
       grid_wait_dependencies();
       for (int i = 0; i < nst && ok; ++i) {
         // scales: issue octet o at the first stage that touches group 8*o

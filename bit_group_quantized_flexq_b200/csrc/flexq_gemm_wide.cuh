@@ -187,6 +187,17 @@ __global__ void __launch_bounds__(WideCfg::kThreads, 1)
     }
     mbar_init(&ctrl->done, 1);
     fence_barrier_init();
+    // weights are read-only inputs: the first ring's worth is requested at
+    // once, before the TMEM allocation and before waiting for the kernel
+    // that produced the activations
+    const int n_pre = nst < STAGES ? nst : STAGES;
+    for (int i = 0; i < n_pre; ++i) {
+      if (args.stall && i == 0) continue;
+      mbar_arrive_expect_tx(&ctrl->full[i], Cfg::kStageBytes);
+      bulk_load(w_ring + i * Cfg::kWStageBytes,
+                args.wp + (static_cast<size_t>(nt) * KB + kb0 + 2 * i) * kWTileBytes,
+                Cfg::kWStageBytes, &ctrl->full[i]);
+    }
     prefetch_tensormap(&tmap_x);
   }
   if (warp == 1) tmem_alloc(&ctrl->tmem_base, Cfg::kTmemCols);
@@ -234,16 +245,8 @@ __global__ void __launch_bounds__(WideCfg::kThreads, 1)
       if (lane == 0) {
         uint32_t issued = 0, parity = 0;
         bool ok = true;
-        // weights are read-only inputs: the first ring's worth is requested
-        // before waiting for the kernel that produced the activations
+        // the first ring's weights were requested during set-up
         const int n_pre = nst < STAGES ? nst : STAGES;
-        for (int i = 0; i < n_pre; ++i) {
-          if (args.stall && i == 0) continue;
-          mbar_arrive_expect_tx(&ctrl->full[i], Cfg::kStageBytes);
-          bulk_load(w_ring + i * Cfg::kWStageBytes,
-                    args.wp + (static_cast<size_t>(nt) * KB + kb0 + 2 * i) * kWTileBytes,
-                    Cfg::kWStageBytes, &ctrl->full[i]);
-        }
         grid_wait_dependencies();
         for (int i = 0; i < nst; ++i) {
           const int s = i % STAGES;
