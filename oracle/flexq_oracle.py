@@ -216,6 +216,83 @@ def unpack_device_form(dev, N, K):
 
 
 # --------------------------------------------------------------------------
+# the "4+2" bit-plane form (after the split storage of 6-bit values into a
+# 4-bit and a 2-bit part, ZeroQuant(4+2) abstract): each code's top four
+# bits go to a 4-bit plane, its low two bits to a 2-bit plane
+# --------------------------------------------------------------------------
+def pack_planes42(codes16):
+    """The 4-bit and the 2-bit plane of one 16-code block.
+
+    codes16: int array [..., 16] of 6-bit codes in [-32, 31]; u_j = c_j & 63,
+    h_j = u_j >> 2 (bits 5:2), l_j = u_j & 3 (bits 1:0).
+    4-bit plane, 8 bytes: byte t (t = 0..3) holds h_t in its high nibble and
+      h_{4+t} in its low nibble; byte 4+t holds h_{8+t} high, h_{12+t} low.
+    2-bit plane, 4 bytes: byte t holds l_t in bits 1:0, l_{4+t} in bits 3:2,
+      l_{8+t} in bits 5:4 and l_{12+t} in bits 7:6.
+    Returns (nibble bytes uint8 [..., 8], two-bit bytes uint8 [..., 4]).
+    """
+    c = np.asarray(codes16)
+    assert c.shape[-1] == BLOCK
+    assert c.min(initial=0) >= -32 and c.max(initial=0) <= 31
+    u = c.astype(np.int64) & 0x3F
+    h, l = u >> 2, u & 3
+    nib = np.zeros(c.shape[:-1] + (8,), dtype=np.int64)
+    two = np.zeros(c.shape[:-1] + (4,), dtype=np.int64)
+    for t in range(4):
+        nib[..., t] = (h[..., t] << 4) | h[..., 4 + t]
+        nib[..., 4 + t] = (h[..., 8 + t] << 4) | h[..., 12 + t]
+        two[..., t] = l[..., t] | (l[..., 4 + t] << 2) | (l[..., 8 + t] << 4) | (l[..., 12 + t] << 6)
+    return nib.astype(np.uint8), two.astype(np.uint8)
+
+
+def unpack_planes42(nib, two):
+    """Inverse of pack_planes42: (uint8 [..., 8], uint8 [..., 4]) -> int8 [..., 16]."""
+    nib = np.asarray(nib).astype(np.int64)
+    two = np.asarray(two).astype(np.int64)
+    u = np.zeros(nib.shape[:-1] + (BLOCK,), dtype=np.int64)
+    for t in range(4):
+        u[..., t] = ((nib[..., t] >> 4) << 2) | (two[..., t] & 3)
+        u[..., 4 + t] = ((nib[..., t] & 15) << 2) | ((two[..., t] >> 2) & 3)
+        u[..., 8 + t] = ((nib[..., 4 + t] >> 4) << 2) | ((two[..., t] >> 4) & 3)
+        u[..., 12 + t] = ((nib[..., 4 + t] & 15) << 2) | ((two[..., t] >> 6) & 3)
+    return (u - 64 * (u >= 32)).astype(np.int8)
+
+
+def pack_device_form42(codes):
+    """6-bit codes [N, K] (N % 128 == 0, K % 128 == 0) -> "4+2" device bytes.
+
+    Tiles as in pack_device_form: tile (nt, kb) (rows nt*128 .. nt*128+127,
+    codes kb*128 .. kb*128+127) is 12288 contiguous bytes at offset
+    (nt*(K/128) + kb) * 12288.  Inside a tile the 4-bit plane comes first:
+    byte b of 16-byte chunk j (j = 0..3) of row r at (j*128 + r)*16 + b, where
+    a row's 64 nibble bytes are its eight blocks' 8-byte nibble planes in
+    order; then the 2-bit plane: chunk 4 + j (j = 0, 1) holds the row's 32
+    two-bit bytes, the eight blocks' 4-byte planes in order.  Each plane is a
+    contiguous, 16-byte aligned 8192- (4-bit) or 4096-byte (2-bit) region of
+    the tile.
+    """
+    codes = np.asarray(codes)
+    N, K = codes.shape
+    assert N % TILE_ROWS == 0 and K % TILE_K == 0
+    nib, two = pack_planes42(codes.reshape(N, K // BLOCK, BLOCK))      # [N, K/16, 8|4]
+    NT, KB = N // TILE_ROWS, K // TILE_K
+    nib_rows = nib.reshape(NT, TILE_ROWS, KB, 4, CHUNK)                # 64 B per row and tile
+    two_rows = two.reshape(NT, TILE_ROWS, KB, 2, CHUNK)                # 32 B per row and tile
+    chunks = np.concatenate([nib_rows, two_rows], axis=3)              # [NT, 128, KB, 6, 16]
+    return np.ascontiguousarray(chunks.transpose(0, 2, 3, 1, 4)).reshape(-1)
+
+
+def unpack_device_form42(dev, N, K):
+    """Inverse of pack_device_form42: "4+2" device bytes -> int8 codes [N, K]."""
+    NT, KB = N // TILE_ROWS, K // TILE_K
+    v = np.asarray(dev, dtype=np.uint8).reshape(NT, KB, 6, TILE_ROWS, CHUNK)
+    rows = np.ascontiguousarray(v.transpose(0, 3, 1, 2, 4))            # [NT, 128, KB, 6, 16]
+    nib = rows[:, :, :, :4, :].reshape(N, K // BLOCK, 8)
+    two = rows[:, :, :, 4:, :].reshape(N, K // BLOCK, 4)
+    return unpack_planes42(nib, two).reshape(N, K)
+
+
+# --------------------------------------------------------------------------
 # the GEMM: exact per-group integer partials, FP64 rescale, one FP16 rounding
 # --------------------------------------------------------------------------
 def group_partials(qa, qw, gs):

@@ -321,6 +321,87 @@ def test_device_form_tile_positions():
                 assert dev[off] == row_bytes[pos], (n, b, pos)
 
 
+# --------------------------------------------------- "4+2" bit planes ------
+def _block42_codes(spec):
+    c = np.zeros(16, dtype=np.int8)
+    if spec == "all -1":
+        c[:] = -1
+    elif spec == "all 1":
+        c[:] = 1
+    else:
+        for j, v in spec.items():
+            c[int(j)] = v
+    return c
+
+
+def test_planes42_hand_worked_cases(golden_dir):
+    g = _golden("planes42_cases.json", golden_dir)
+    for case in g["cases"]:
+        codes = _block42_codes(case["codes"])
+        nib, two = orc.pack_planes42(codes)
+        assert nib.tobytes().hex() == case["nib"], case
+        assert two.tobytes().hex() == case["two"], case
+        assert np.array_equal(orc.unpack_planes42(nib, two), codes)
+
+
+def test_planes42_is_a_bit_permutation():
+    # one bit of one code's 6-bit field sets exactly one of the block's 96
+    # bits, and the 96 (code, bit) pairs land on 96 distinct bits
+    seen = set()
+    for j in range(16):
+        for bit in range(6):
+            u = 1 << bit
+            c = np.zeros(16, dtype=np.int8)
+            c[j] = u - 64 if u >= 32 else u
+            nib, two = orc.pack_planes42(c)
+            value = int.from_bytes(nib.tobytes() + two.tobytes(), "little")
+            assert bin(value).count("1") == 1, (j, bit)
+            seen.add(value.bit_length() - 1)
+    assert seen == set(range(96))
+    # the high four bits of a code go to the 4-bit plane, the low two to the 2-bit plane
+    for j in range(16):
+        nib, two = orc.pack_planes42(np.eye(16, dtype=np.int8)[j] * 3)          # u = 0b000011
+        assert not nib.any() and two.any()
+        nib, two = orc.pack_planes42(np.eye(16, dtype=np.int8)[j] * -4)         # u = 0b111100
+        assert nib.any() and not two.any()
+
+
+def test_planes42_roundtrip_every_value_at_every_position():
+    rng = np.random.default_rng(14)
+    base = rng.integers(-32, 32, (64, 16)).astype(np.int8)
+    for j in range(16):
+        c = base.copy()
+        c[:, j] = np.arange(-32, 32, dtype=np.int8)
+        assert np.array_equal(orc.unpack_planes42(*orc.pack_planes42(c)), c)
+
+
+def test_device_form42_tile_positions():
+    N, K = 256, 384
+    rng = np.random.default_rng(19)
+    codes = rng.integers(-32, 32, (N, K)).astype(np.int8)
+    dev = orc.pack_device_form42(codes)
+    assert dev.size == N * K * 3 // 4
+    assert np.array_equal(orc.unpack_device_form42(dev, N, K), codes)
+    KB = K // 128
+    for n in (0, 1, 127, 128, 200, 255):
+        nt, r = divmod(n, 128)
+        for b in (0, 5, 7, 8, 15, 23):
+            nib, two = orc.pack_planes42(codes[n, 16 * b:16 * b + 16])
+            kb, bt = divmod(b, 8)                  # tile along K, block within the tile
+            tile = (nt * KB + kb) * 12288
+            for pos in range(8):                   # 4-bit plane: row byte 8*bt + pos, chunks 0..3
+                j, byte = divmod(8 * bt + pos, 16)
+                assert dev[tile + (j * 128 + r) * 16 + byte] == nib[pos], (n, b, pos)
+            for pos in range(4):                   # 2-bit plane: row byte 4*bt + pos, chunks 4, 5
+                j, byte = divmod(4 * bt + pos, 16)
+                assert dev[tile + ((4 + j) * 128 + r) * 16 + byte] == two[pos], (n, b, pos)
+    # the planes are contiguous regions of each tile
+    t0 = dev[:12288].reshape(6, 128, 16)
+    nib_rows = t0[:4].transpose(1, 0, 2).reshape(128, 64)
+    assert np.array_equal(nib_rows[3], np.concatenate(
+        [orc.pack_planes42(codes[3, 16 * b:16 * b + 16])[0] for b in range(8)]))
+
+
 # ------------------------------------------------------------ GEMM ----------
 def test_gemm_hand_worked_case(golden_dir):
     g = _golden("gemm_case.json", golden_dir)
