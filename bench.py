@@ -547,6 +547,7 @@ def run_flexq(args, rank, world):
         result["act_quant"] = act_quant_diagnostics(device, hbm)
         result["mixed_stack"] = stack_diagnostics(device, hbm, int8_peak)
         result["other_configs"] = run_sweep(device, hbm, int8_peak, subset=True)
+        result["layout_ab"] = layout_ab(device, hbm)
     if args.e2e:
         result["e2e"] = run_e2e(W, args, device, world)
     if rank == 0 and world == 1 and args.cpu_baseline:
@@ -794,6 +795,55 @@ def run_sweep(device, hbm_gbs, int8_peak_tops, subset=False):
         del copies
         torch.cuda.empty_cache()
     return out
+
+
+def layout_ab(device, hbm_gbs, ms=(1, 16)):
+    """A/B of the two packed-weight layouts at decode sizes on the three
+    LLaMA-2-70B layer shapes of the step: the byte-aligned device form and
+    the "4+2" bit-plane form hold the same codes and run the same kernels,
+    only the unpack differs.  Per (shape, M, layout): the GEMM alone on
+    quantized activations and the whole layer, device time per call from a
+    CUDA graph rotating over enough weight copies to exceed L2, and the
+    fraction of the HBM roofline; `ratio` = byte-aligned time / 4+2 time
+    (above 1: 4+2 faster)."""
+    import torch
+    from bit_group_quantized_flexq_b200 import flexq, inputs
+    stream = torch.cuda.Stream(device)
+    rows = []
+    for (N, K, bits) in ((8192, 8192, 6), (28672, 8192, 6), (8192, 28672, 8)):
+        w = inputs.weights(N, K, std=WEIGHT_STD, seed=inputs.layer_seed("ab", N, K), device=device)
+        n_copies = max(2, int((400 << 20) // (N * K * 3 // 4)) + 1)
+        packed = {lay: [flexq.quantize_weight(w, GS, layout=lay) for _ in range(n_copies)]
+                  for lay in (flexq.LAYOUT_BYTE_ALIGNED, flexq.LAYOUT_4_2)}
+        del w
+        for M in ms:
+            x = inputs.activations(M, K, outlier_frac=OUTLIER_FRAC, outlier_scale=OUTLIER_SCALE,
+                                   seed=inputs.layer_seed("ab-x", M, K)).to(device)
+            xq, xs = flexq.quantize_act(x, GS, bits)
+            y = torch.empty(M, N, dtype=torch.float16, device=device)
+            row = {"M": M, "N": N, "K": K, "act_bits": bits}
+            for lay, name in ((flexq.LAYOUT_BYTE_ALIGNED, "byte_aligned"), (flexq.LAYOUT_4_2, "4+2")):
+                cps = packed[lay]
+
+                def g_body(cps=cps, lay=lay):
+                    for wp, ws in cps:
+                        flexq.gemm(xq, xs, wp, ws, N, GS, bits, out=y, layout=lay)
+
+                def l_body(cps=cps, lay=lay):
+                    for wp, ws in cps:
+                        flexq.linear(x, wp, ws, N, GS, bits, out=y, layout=lay)
+                g_us = _graph_time_us(g_body, device, stream, 3) / len(cps)
+                l_us = _graph_time_us(l_body, device, stream, 3) / len(cps)
+                row[f"{name}_gemm_us"] = round(g_us, 2)
+                row[f"{name}_gemm_frac_hbm"] = round(gemm_bytes(M, N, K) / (g_us * 1e-6) / 1e9 / hbm_gbs, 4)
+                row[f"{name}_linear_us"] = round(l_us, 2)
+            row["ratio_gemm"] = round(row["byte_aligned_gemm_us"] / row["4+2_gemm_us"], 4)
+            row["ratio_linear"] = round(row["byte_aligned_linear_us"] / row["4+2_linear_us"], 4)
+            rows.append(row)
+            del x, xq, xs, y
+        del packed
+        torch.cuda.empty_cache()
+    return rows
 
 
 def int8_library_context(W, device, M, reps=20):

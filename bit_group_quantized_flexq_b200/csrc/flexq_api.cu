@@ -64,7 +64,7 @@ struct DeviceState {
   bool ready = false;
   int sms = 148;
   unsigned int* status = nullptr;
-  unsigned attr_mask = 0;        // which GEMM instantiations got their smem limit
+  unsigned long long attr_mask = 0;   // which GEMM instantiations got their smem limit
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -284,14 +284,14 @@ int smem_bytes_for() {
   return 1024 + ctrl_offset_for<T>() + static_cast<int>(sizeof(flexq::GemmCtrl<T>));
 }
 
-template <int T, bool PARTIALS, bool FUSEDQ = false>
+template <int T, bool PARTIALS, bool FUSEDQ = false, int LAYOUT = 0>
 int launch_gemm_t(DeviceState* st, const CUtensorMap& map, const CUtensorMap& map_sa,
                   const flexq::LayerTable& tab, flexq::GemmArgs a, long long grid_ctas,
                   cudaStream_t stream) {
   using Cfg = flexq::GemmCfg<T>;
-  auto kern = flexq::gemm_w6ax_kernel<T, PARTIALS, FUSEDQ>;
-  const unsigned bit = 1u << ((T == 16 ? 0 : T == 32 ? 1 : T == 64 ? 2 : 3) + (PARTIALS ? 4 : 0) +
-                              (FUSEDQ ? 8 : 0));
+  auto kern = flexq::gemm_w6ax_kernel<T, PARTIALS, FUSEDQ, LAYOUT>;
+  const unsigned long long bit =
+      1ull << ((T == 16 ? 0 : T == 32 ? 1 : 2) + (PARTIALS ? 4 : 0) + (FUSEDQ ? 8 : 0) + 16 * LAYOUT);
   const int smem = smem_bytes_for<T, FUSEDQ>();
   {
     std::lock_guard<std::mutex> lock(g_dev_mutex);
@@ -341,12 +341,12 @@ flexq::LayerTable single_layer_table(const CUtensorMap& map_sw, const void* Wp, 
 }
 
 // 128-token tiles: the warpgroup-role kernel of flexq_gemm_wide.cuh.
-template <bool PARTIALS>
+template <bool PARTIALS, int LAYOUT = 0>
 int launch_gemm_wide(DeviceState* st, const CUtensorMap& map, flexq::GemmArgs a,
                      long long grid_ctas, cudaStream_t stream) {
   using Cfg = flexq::WideCfg;
-  auto kern = flexq::gemm_w6ax_wide_kernel<PARTIALS>;
-  const unsigned bit = 1u << (12 + (PARTIALS ? 1 : 0));
+  auto kern = flexq::gemm_w6ax_wide_kernel<PARTIALS, LAYOUT>;
+  const unsigned long long bit = 1ull << (32 + (PARTIALS ? 1 : 0) + 2 * LAYOUT);
   const int ctrl_off = (Cfg::kMainBytes + 15) & ~15;
   const int smem = 1024 + ctrl_off + static_cast<int>(sizeof(flexq::WideCtrl));
   {
@@ -409,7 +409,7 @@ int apply_workspace(Plan* plan, int M, int N, void* workspace, size_t workspace_
 
 int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, const void* Wp,
                 const void* Ws, void* Y, int32_t* P, bool partials, void* workspace,
-                size_t workspace_bytes, void* stream) {
+                size_t workspace_bytes, void* stream, int layout = 0) {
   int rc = check_gemm_shape(M, N, K, gs);
   if (rc) return rc;
   if (M == 0) return ok();               // empty batch: nothing to read or write
@@ -455,6 +455,15 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
   a.stall = g_inject_stall.exchange(0);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const flexq::LayerTable tab = single_layer_table(map_sw, Wp, Y, N, plan);
+  if (layout == 1 && !partials) {
+    switch (plan.T) {
+      case 16: rc = launch_gemm_t<16, false, false, 1>(st, map, map_sa, tab, a, plan.ctas, s); break;
+      case 32: rc = launch_gemm_t<32, false, false, 1>(st, map, map_sa, tab, a, plan.ctas, s); break;
+      case 64: rc = launch_gemm_t<64, false, false, 1>(st, map, map_sa, tab, a, plan.ctas, s); break;
+      default: rc = launch_gemm_wide<false, 1>(st, map, a, plan.ctas, s); break;
+    }
+    return rc ? rc : ok();
+  }
   switch (plan.T) {
     case 16: rc = partials ? launch_gemm_t<16, true>(st, map, map_sa, tab, a, plan.ctas, s) : launch_gemm_t<16, false>(st, map, map_sa, tab, a, plan.ctas, s); break;
     case 32: rc = partials ? launch_gemm_t<32, true>(st, map, map_sa, tab, a, plan.ctas, s) : launch_gemm_t<32, false>(st, map, map_sa, tab, a, plan.ctas, s); break;
@@ -507,7 +516,8 @@ LinearLayout linear_layout(const Plan& p, int M, int N, int K, int gs) {
 }
 
 int linear_common(int M, int N, int K, int gs, int bits, const void* X, const void* Wp,
-                  const void* Ws, void* Y, void* workspace, size_t workspace_bytes, void* stream) {
+                  const void* Ws, void* Y, void* workspace, size_t workspace_bytes, void* stream,
+                  int layout = 0) {
   if (bits != 6 && bits != 8) return fail(FLEXQ_ERR_INVALID_ARG, "bits=%d is not 6 or 8", bits);
   int rc = check_gemm_shape(M, N, K, gs);
   if (rc) return rc;
@@ -529,7 +539,7 @@ int linear_common(int M, int N, int K, int gs, int bits, const void* X, const vo
     void* xs = static_cast<char*>(workspace) + L.xs_off;
     if ((rc = flexq_quantize_act(M, K, gs, bits, X, xq, xs, stream))) return rc;
     return gemm_common(M, N, K, gs, xq, xs, Wp, Ws, Y, nullptr, false, workspace, L.xq_off,
-                       stream);
+                       stream, layout);
   }
   if ((rc = apply_workspace(&plan, M, N, workspace, workspace_bytes))) return rc;
   CUtensorMap map_x, map_sa, map_sw;     // activations and their scales: read by the kernel itself
@@ -553,8 +563,12 @@ int linear_common(int M, int N, int K, int gs, int bits, const void* X, const vo
   a.split = plan.split;
   a.stall = g_inject_stall.exchange(0);
   const flexq::LayerTable tab = single_layer_table(map_sw, Wp, Y, N, plan);
-  rc = launch_gemm_t<16, false, true>(st, map_x, map_sa, tab, a, plan.ctas,
-                                      static_cast<cudaStream_t>(stream));
+  if (layout == 1)
+    rc = launch_gemm_t<16, false, true, 1>(st, map_x, map_sa, tab, a, plan.ctas,
+                                           static_cast<cudaStream_t>(stream));
+  else
+    rc = launch_gemm_t<16, false, true>(st, map_x, map_sa, tab, a, plan.ctas,
+                                        static_cast<cudaStream_t>(stream));
   return rc ? rc : ok();
 }
 
@@ -844,6 +858,14 @@ size_t flexq_weight_packed_bytes(int N, int K, int group_size) {
 
 int flexq_quantize_weight(int N, int K, int group_size, const void* W_fp16, void* Wq_packed,
                           void* W_scales_fp16, void* stream) {
+  return flexq_quantize_weight_layout(N, K, group_size, FLEXQ_LAYOUT_BYTE_ALIGNED, W_fp16,
+                                      Wq_packed, W_scales_fp16, stream);
+}
+
+int flexq_quantize_weight_layout(int N, int K, int group_size, int layout, const void* W_fp16,
+                                 void* Wq_packed, void* W_scales_fp16, void* stream) {
+  if (layout != FLEXQ_LAYOUT_BYTE_ALIGNED && layout != FLEXQ_LAYOUT_4_2)
+    return fail(FLEXQ_ERR_INVALID_ARG, "layout=%d is not a weight layout", layout);
   int rc = check_gemm_shape(1, N, K, group_size);
   if (rc) return rc;
   const void* ptrs[] = {W_fp16, Wq_packed, W_scales_fp16};
@@ -857,9 +879,14 @@ int flexq_quantize_weight(int N, int K, int group_size, const void* W_fp16, void
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "weight_scale_kernel launch");
   const long long n2 = static_cast<long long>(N) * (K / 128) * 2;
-  flexq::weight_pack_kernel<<<static_cast<unsigned>((n2 + 255) / 256), 256, 0, s>>>(
-      static_cast<const __half*>(W_fp16), static_cast<const __half*>(W_scales_fp16),
-      static_cast<uint8_t*>(Wq_packed), N, K, group_size);
+  if (layout == FLEXQ_LAYOUT_4_2)
+    flexq::weight_pack42_kernel<<<static_cast<unsigned>((n2 + 255) / 256), 256, 0, s>>>(
+        static_cast<const __half*>(W_fp16), static_cast<const __half*>(W_scales_fp16),
+        static_cast<uint8_t*>(Wq_packed), N, K, group_size);
+  else
+    flexq::weight_pack_kernel<<<static_cast<unsigned>((n2 + 255) / 256), 256, 0, s>>>(
+        static_cast<const __half*>(W_fp16), static_cast<const __half*>(W_scales_fp16),
+        static_cast<uint8_t*>(Wq_packed), N, K, group_size);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "weight_pack_kernel launch");
   return ok();
@@ -1016,6 +1043,27 @@ int flexq_linear_w6a8(int M, int N, int K, int group_size, const void* X_fp16,
                       size_t workspace_bytes, void* stream) {
   return linear_common(M, N, K, group_size, 8, X_fp16, Wq_packed, W_scales, Y_fp16, workspace,
                        workspace_bytes, stream);
+}
+
+int flexq_gemm_layout(int M, int N, int K, int group_size, int act_bits, int layout,
+                      const int8_t* Xq, const void* X_scales, const void* Wq_packed,
+                      const void* W_scales, void* Y_fp16, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  if (act_bits != 6 && act_bits != 8)
+    return fail(FLEXQ_ERR_INVALID_ARG, "act_bits=%d is not 6 or 8", act_bits);
+  if (layout != FLEXQ_LAYOUT_BYTE_ALIGNED && layout != FLEXQ_LAYOUT_4_2)
+    return fail(FLEXQ_ERR_INVALID_ARG, "layout=%d is not a weight layout", layout);
+  return gemm_common(M, N, K, group_size, Xq, X_scales, Wq_packed, W_scales, Y_fp16, nullptr,
+                     false, workspace, workspace_bytes, stream, layout);
+}
+
+int flexq_linear_layout(int M, int N, int K, int group_size, int act_bits, int layout,
+                        const void* X_fp16, const void* Wq_packed, const void* W_scales,
+                        void* Y_fp16, void* workspace, size_t workspace_bytes, void* stream) {
+  if (layout != FLEXQ_LAYOUT_BYTE_ALIGNED && layout != FLEXQ_LAYOUT_4_2)
+    return fail(FLEXQ_ERR_INVALID_ARG, "layout=%d is not a weight layout", layout);
+  return linear_common(M, N, K, group_size, act_bits, X_fp16, Wq_packed, W_scales, Y_fp16,
+                       workspace, workspace_bytes, stream, layout);
 }
 
 int flexq_debug_check_quantizer(unsigned long long* mismatches, unsigned int* first_mismatch) {

@@ -248,6 +248,31 @@ __device__ __forceinline__ void unpack_block(uint32_t w0, uint32_t w1, uint32_t 
   out[3] = ((p2 * 4u + p1) * 4u + p0) * 4u;
 }
 
+// One 16-code block of the "4+2" form (nibble words n0, n1 and the 2-bit
+// word l, see weight_pack42_kernel) -> four int8x4 words in k order, each
+// byte code * 4 = h << 4 | l << 2: the nibbles in bits 7:4, the 2-bit pieces
+// shifted into bits 3:2.
+__device__ __forceinline__ void unpack_block42(uint32_t n0, uint32_t n1, uint32_t l,
+                                               uint32_t* out) {
+  out[0] = (n0 & 0xF0F0F0F0u) | ((l << 2) & 0x0C0C0C0Cu);
+  out[1] = ((n0 << 4) & 0xF0F0F0F0u) | (l & 0x0C0C0C0Cu);
+  out[2] = (n1 & 0xF0F0F0F0u) | ((l >> 2) & 0x0C0C0C0Cu);
+  out[3] = ((n1 << 4) & 0xF0F0F0F0u) | ((l >> 4) & 0x0C0C0C0Cu);
+}
+
+// The 24 words of one row's 96 packed bytes of a 128-code tile (six 16-byte
+// chunks) -> its 128 int8 codes * 4, in k order, for either weight layout.
+template <int LAYOUT>
+__device__ __forceinline__ void unpack_row_tile(const uint32_t (&w)[24], uint32_t (&out)[32]) {
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    if (LAYOUT == 0)
+      unpack_block(w[3 * b], w[3 * b + 1], w[3 * b + 2], &out[4 * b]);
+    else
+      unpack_block42(w[2 * b], w[2 * b + 1], w[16 + b], &out[4 * b]);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Fused activation quantization (FUSEDQ, token tiles of 16 rows): the kernel
 // reads the FP16 activations itself.  At stage i unpack warp q quantizes rows
@@ -354,7 +379,7 @@ __device__ __forceinline__ void quantize_act_rows(uint4 (&xv)[R], int Mt, int m0
   }
 }
 
-template <int T, bool PARTIALS, bool FUSEDQ = false>
+template <int T, bool PARTIALS, bool FUSEDQ = false, int LAYOUT = 0>
 __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     gemm_w6ax_kernel(const __grid_constant__ CUtensorMap tmap_x,
                      const __grid_constant__ CUtensorMap tmap_sa,
@@ -703,8 +728,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
           if (lane == 0) mbar_arrive(&ctrl->empty[st.idx]);
         }
         uint32_t out[32];
-#pragma unroll
-        for (int b = 0; b < 8; ++b) unpack_block(w[3 * b], w[3 * b + 1], w[3 * b + 2], &out[4 * b]);
+        unpack_row_tile<LAYOUT>(w, out);
         tmem_st32(col + 32 * t, out);
       }
       tmem_wait_st();

@@ -122,7 +122,7 @@ __device__ __forceinline__ void wide_store_partials(const uint32_t (&pv)[32], in
   }
 }
 
-template <bool PARTIALS>
+template <bool PARTIALS, int LAYOUT = 0>
 __global__ void __launch_bounds__(WideCfg::kThreads, 1)
     gemm_w6ax_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
   using Cfg = WideCfg;
@@ -405,8 +405,7 @@ __global__ void __launch_bounds__(WideCfg::kThreads, 1)
           if (lane == 0) mbar_arrive(&ctrl->empty[st.idx]);
         }
         uint32_t out[32];
-#pragma unroll
-        for (int b = 0; b < 8; ++b) unpack_block(w[3 * b], w[3 * b + 1], w[3 * b + 2], &out[4 * b]);
+        unpack_row_tile<LAYOUT>(w, out);
         tmem_st32(col + 32 * t, out);
       }
       tmem_wait_st();

@@ -283,6 +283,74 @@ __global__ void __launch_bounds__(256) weight_pack_kernel(
 }
 
 // --------------------------------------------------------------------------
+// The "4+2" bit-plane form (layout 1): the top four bits h of each 6-bit code
+// u go to a 4-bit plane, the low two bits l to a 2-bit plane.  Per 16-code
+// block: nibble words N0, N1 (byte t of N0 = h_t << 4 | h_{4+t}, byte t of
+// N1 = h_{8+t} << 4 | h_{12+t}) and one 2-bit word L (byte t = l_t |
+// l_{4+t} << 2 | l_{8+t} << 4 | l_{12+t} << 6).  Tiles as in the byte-aligned
+// form; inside a tile, chunks 0..3 of each row are its nibble plane (block b
+// at row bytes 8b..8b+7) and chunks 4, 5 its 2-bit plane (block b at row
+// bytes 4b..4b+3): each plane is one contiguous 16-byte aligned region.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void pack_block42(const uint32_t (&u)[16], uint32_t& n0, uint32_t& n1,
+                                             uint32_t& l) {
+  n0 = n1 = l = 0u;
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    n0 |= (((u[t] >> 2) << 4) | (u[4 + t] >> 2)) << (8 * t);
+    n1 |= (((u[8 + t] >> 2) << 4) | (u[12 + t] >> 2)) << (8 * t);
+    l |= ((u[t] & 3u) | ((u[4 + t] & 3u) << 2) | ((u[8 + t] & 3u) << 4) | ((u[12 + t] & 3u) << 6))
+         << (8 * t);
+  }
+}
+
+// Weight quantization, pass 2 for the "4+2" form: one thread per (row n,
+// 64-code half of a 128-code K-block): four blocks, i.e. two 16-byte chunks
+// of the nibble plane and one of the 2-bit plane.
+__global__ void __launch_bounds__(256) weight_pack42_kernel(
+    const __half* __restrict__ W, const __half* __restrict__ Ws,
+    uint8_t* __restrict__ Wp, int N, int K, int gs) {
+  const int KB = K / 128;
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= static_cast<long long>(N) * KB * 2) return;
+  const int half_idx = static_cast<int>(t & 1);
+  const long long nk = t >> 1;
+  const int n = static_cast<int>(nk / KB);
+  const int kb = static_cast<int>(nk - static_cast<long long>(n) * KB);
+  const int k0 = kb * 128 + half_idx * 64;
+  const uint4* p = reinterpret_cast<const uint4*>(W + static_cast<long long>(n) * K + k0);
+  uint32_t nib[8], two[4];
+#pragma unroll
+  for (int blk = 0; blk < 4; ++blk) {
+    uint32_t u[16];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint4 raw = __ldg(p + 2 * blk + c);
+      const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+      const int kk = k0 + 16 * blk + 8 * c;
+      const float s = __half2float(Ws[static_cast<long long>(kk / gs) * N + n]);
+      const float rs = s == 0.0f ? 0.0f : __frcp_rn(s);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h2[i]);
+        u[8 * c + 2 * i] = static_cast<uint32_t>(quant_code(f.x, s, rs, 31)) & 0x3Fu;
+        u[8 * c + 2 * i + 1] = static_cast<uint32_t>(quant_code(f.y, s, rs, 31)) & 0x3Fu;
+      }
+    }
+    pack_block42(u, nib[2 * blk], nib[2 * blk + 1], two[blk]);
+  }
+  const int nt = n >> 7, r = n & 127;
+  uint8_t* tile = Wp + (static_cast<long long>(nt) * KB + kb) * 12288;
+#pragma unroll
+  for (int jj = 0; jj < 2; ++jj) {              // nibble chunks 2h, 2h + 1
+    uint4* dst = reinterpret_cast<uint4*>(tile + ((2 * half_idx + jj) * 128 + r) * 16);
+    *dst = make_uint4(nib[4 * jj], nib[4 * jj + 1], nib[4 * jj + 2], nib[4 * jj + 3]);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(tile + ((4 + half_idx) * 128 + r) * 16);
+  *dst = make_uint4(two[0], two[1], two[2], two[3]);
+}
+
+// --------------------------------------------------------------------------
 // Test hook: for FP16 scale patterns [s_first, s_first + n_s) (positive,
 // finite) against every finite FP16 value x, for Q = 31 and Q = 127, counts
 // the (x, s) pairs where a route of the quantizers differs from

@@ -23,6 +23,8 @@ FLEXQ_ERR_DEVICE_TIMEOUT = 5
 
 _lib = None
 MAX_GROUP_LAYERS = 4
+LAYOUT_BYTE_ALIGNED = 0      # the default device form of the packed weights
+LAYOUT_4_2 = 1               # the "4+2" bit-plane form
 
 
 class Layer(ctypes.Structure):
@@ -84,6 +86,14 @@ def lib():
             "flexq_set_wait_limit_ns": (c_int, [ctypes.c_uint64]),
             "flexq_debug_inject_stall": (c_int, [c_int]),
             "flexq_get_device_status": (c_int, [c_void_p]),
+            "flexq_quantize_weight_layout": (c_int, [c_int, c_int, c_int, c_int, c_void_p,
+                                                     c_void_p, c_void_p, c_void_p]),
+            "flexq_gemm_layout": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, c_void_p,
+                                          c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                          c_size_t, c_void_p]),
+            "flexq_linear_layout": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, c_void_p,
+                                            c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                            c_void_p]),
             "flexq_gemm_group": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_int,
                                          ctypes.POINTER(Layer), c_void_p, c_size_t, c_void_p]),
             "flexq_linear_group": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_int,
@@ -153,9 +163,9 @@ def weight_scales_view(ws):
     return ws.t()
 
 
-def quantize_weight(w, group_size, out=None):
-    """FP16 W [N, K] -> (packed uint8 [3NK/4] in the device form, FP16 scales
-    stored group-major as a [K/gs, N] tensor)."""
+def quantize_weight(w, group_size, out=None, layout=LAYOUT_BYTE_ALIGNED):
+    """FP16 W [N, K] -> (packed uint8 [3NK/4] in the device form of `layout`,
+    FP16 scales stored group-major as a [K/gs, N] tensor)."""
     _need(w, "w", torch.float16)
     N, K = w.shape
     nbytes = weight_packed_bytes(N, K, group_size)
@@ -167,7 +177,12 @@ def quantize_weight(w, group_size, out=None):
     wp, ws = out
     _need(wp, "packed", torch.uint8, (nbytes,))
     _need(ws, "scales", torch.float16, (K // group_size, N))
-    _check(lib().flexq_quantize_weight(N, K, group_size, _ptr(w), _ptr(wp), _ptr(ws), _stream(w)))
+    if layout == LAYOUT_BYTE_ALIGNED:
+        _check(lib().flexq_quantize_weight(N, K, group_size, _ptr(w), _ptr(wp), _ptr(ws),
+                                           _stream(w)))
+    else:
+        _check(lib().flexq_quantize_weight_layout(N, K, group_size, layout, _ptr(w), _ptr(wp),
+                                                  _ptr(ws), _stream(w)))
     return wp, ws
 
 
@@ -218,7 +233,8 @@ def reset_workspaces():
         t.zero_()
 
 
-def gemm(xq, xs, wp, ws, N, group_size, act_bits=6, out=None, workspace_buf=None):
+def gemm(xq, xs, wp, ws, N, group_size, act_bits=6, out=None, workspace_buf=None,
+         layout=LAYOUT_BYTE_ALIGNED):
     """Y [M, N] FP16 = dequant(xq, xs) . dequant(wp, ws)^T (W6A6 or W6A8).
 
     workspace_buf: a zero-filled uint8 device tensor of at least
@@ -240,6 +256,10 @@ def gemm(xq, xs, wp, ws, N, group_size, act_bits=6, out=None, workspace_buf=None
     else:
         _need(workspace_buf, "workspace", torch.uint8)
         wsp, wsn = _ptr(workspace_buf), workspace_buf.numel()
+    if layout != LAYOUT_BYTE_ALIGNED:
+        _check(lib().flexq_gemm_layout(M, N, K, group_size, act_bits, layout, _ptr(xq), _ptr(xs),
+                                       _ptr(wp), _ptr(ws), _ptr(out), wsp, wsn, _stream(xq)))
+        return out
     fn = {6: lib().flexq_gemm_w6a6, 8: lib().flexq_gemm_w6a8}[act_bits]
     _check(fn(M, N, K, group_size, _ptr(xq), _ptr(xs), _ptr(wp), _ptr(ws), _ptr(out), wsp, wsn,
               _stream(xq)))
@@ -262,7 +282,8 @@ def force_linear_route(route=0):
     _check(lib().flexq_debug_force_linear_route(route))
 
 
-def linear(x, wp, ws, N, group_size, act_bits=6, out=None, workspace_buf=None):
+def linear(x, wp, ws, N, group_size, act_bits=6, out=None, workspace_buf=None,
+           layout=LAYOUT_BYTE_ALIGNED):
     """Y [M, N] FP16 of a quantized linear layer from FP16 activations x
     [M, K]: the activations are quantized to act_bits (6 or 8) by the rule of
     quantize_act, then multiplied with the packed 6-bit weights.  Batches of
@@ -286,6 +307,10 @@ def linear(x, wp, ws, N, group_size, act_bits=6, out=None, workspace_buf=None):
     else:
         _need(workspace_buf, "workspace", torch.uint8)
         wsp, wsn = _ptr(workspace_buf), workspace_buf.numel()
+    if layout != LAYOUT_BYTE_ALIGNED:
+        _check(lib().flexq_linear_layout(M, N, K, group_size, act_bits, layout, _ptr(x), _ptr(wp),
+                                         _ptr(ws), _ptr(out), wsp, wsn, _stream(x)))
+        return out
     fn = {6: lib().flexq_linear_w6a6, 8: lib().flexq_linear_w6a8}[act_bits]
     _check(fn(M, N, K, group_size, _ptr(x), _ptr(wp), _ptr(ws), _ptr(out), wsp, wsn, _stream(x)))
     return out

@@ -97,6 +97,27 @@ int flexq_quantize_weight(int N, int K, int group_size, const void* W_fp16,
                           void* Wq_packed, void* W_scales_fp16, void* stream);
 
 /*
+ * Weight layouts of the packed buffer.  FLEXQ_LAYOUT_BYTE_ALIGNED is the
+ * device form above (the default everywhere).  FLEXQ_LAYOUT_4_2 is the
+ * "4+2" bit-plane form, after the split storage of 6-bit values into a 4-bit
+ * and a 2-bit part (ZeroQuant(4+2) abstract): with h_j = u_j >> 2 and
+ * l_j = u_j & 3, a 16-code block is an 8-byte 4-bit plane (byte t = h_t << 4
+ * | h_{4+t}, byte 4+t = h_{8+t} << 4 | h_{12+t}) and a 4-byte 2-bit plane
+ * (byte t = l_t | l_{4+t} << 2 | l_{8+t} << 4 | l_{12+t} << 6); tiles as
+ * above, and inside a tile chunks 0..3 of each row hold its eight blocks'
+ * 4-bit planes, chunks 4 and 5 their 2-bit planes, so that each plane is one
+ * contiguous 16-byte aligned region (8192 and 4096 bytes) of the tile.  Same
+ * size, same codes and scales; only the bit placement differs.
+ */
+#define FLEXQ_LAYOUT_BYTE_ALIGNED 0
+#define FLEXQ_LAYOUT_4_2 1
+
+/* flexq_quantize_weight with an explicit layout (FLEXQ_ERR_INVALID_ARG for
+ * any other value). */
+int flexq_quantize_weight_layout(int N, int K, int group_size, int layout, const void* W_fp16,
+                                 void* Wq_packed, void* W_scales_fp16, void* stream);
+
+/*
  * flexq_quantize_act -- per-forward activation quantization, 6 or 8 bits.
  * Passage: 6-bit activations, 8-bit ones kept in sensitive layers (arXiv
  * abstract; blog, "Fine-Grained Quantization and Layer Sensitivity").
@@ -249,6 +270,21 @@ int flexq_gemm_static_scratch(int M, int N, int K, int group_size, int act_bits,
                               const int8_t* Xq, const void* X_scales,
                               const void* Wq_packed, const void* W_scales,
                               void* Y_fp16, void* stream);
+
+/*
+ * flexq_gemm_layout / flexq_linear_layout -- flexq_gemm_w6a6/w6a8 and
+ * flexq_linear_w6a6/w6a8 (act_bits 6 or 8) on packed weights of either
+ * layout (the weights must have been packed with the same layout).  Same
+ * arguments, plans, workspaces and results otherwise; FLEXQ_ERR_INVALID_ARG
+ * for an unknown layout or act_bits.
+ */
+int flexq_gemm_layout(int M, int N, int K, int group_size, int act_bits, int layout,
+                      const int8_t* Xq, const void* X_scales, const void* Wq_packed,
+                      const void* W_scales, void* Y_fp16, void* workspace, size_t workspace_bytes,
+                      void* stream);
+int flexq_linear_layout(int M, int N, int K, int group_size, int act_bits, int layout,
+                        const void* X_fp16, const void* Wq_packed, const void* W_scales,
+                        void* Y_fp16, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * One layer of a grouped call: layers that read the same activations (the

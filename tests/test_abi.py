@@ -209,3 +209,21 @@ def test_group_plan_is_host_only_and_sane(L):
     assert flexq.group_plan(512, 8192, 128, [28672, 28672]) == (128, 0, 0, 3)
     assert flexq.gemm_group_workspace_bytes(1, 8192, 128, [8192, 1024, 1024]) == \
         4096 + 80 * 3 * 16 * 128 * 4
+
+
+def test_layout_validation_before_any_launch(L):
+    assert L.flexq_quantize_weight_layout(128, 256, 128, 2, FAKE, FAKE, FAKE, NULL) == \
+        flexq.FLEXQ_ERR_INVALID_ARG
+    assert L.flexq_quantize_weight_layout(128, 256, 128, 1, FAKE, NULL, FAKE, NULL) == \
+        flexq.FLEXQ_ERR_INVALID_ARG
+    g = L.flexq_gemm_layout
+    assert g(4, 256, 256, 128, 6, 3, FAKE, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == \
+        flexq.FLEXQ_ERR_INVALID_ARG
+    assert g(4, 256, 256, 128, 5, 1, FAKE, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == \
+        flexq.FLEXQ_ERR_INVALID_ARG
+    assert g(4, 200, 256, 128, 6, 1, FAKE, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == \
+        flexq.FLEXQ_ERR_UNSUPPORTED
+    f = L.flexq_linear_layout
+    assert f(4, 256, 256, 128, 6, -1, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == \
+        flexq.FLEXQ_ERR_INVALID_ARG
+    assert f(0, 256, 256, 128, 6, 1, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == flexq.FLEXQ_OK
