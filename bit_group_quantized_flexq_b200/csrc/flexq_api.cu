@@ -477,21 +477,24 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
 // A linear layer from FP16 activations: quantize them (bits 6 or 8), then the
 // group GEMM, in one of two routes.  Inside the GEMM (16-token tiles, one
 // launch) the quantization saves the separate quantizer's launch and its
-// dependency (about 1.4 us per layer) but lengthens every pipeline stage of
-// the unpack warps, by more the more tokens there are; it is taken where
-// each CTA streams few stages: at most 4 stages of K for up to 4 tokens, at
-// most 2 for up to 8 tokens (measured per layer, weights cold: 4096^2 and
-// 1024x8192 layers gain 8-14 % at one token, layers with 6 stages per CTA
-// lose 2-3 %).  Otherwise the activation quantizer runs first, its codes
-// and scales in the caller's workspace after the GEMM's region, whose
-// arrival counters keep their fixed place at the start.
-bool linear_fused(const Plan& p, int M, int K) {
+// dependency (about 1.5 us per layer) but adds the quantization of the
+// tile's rows to every pipeline stage of the unpack warps, a cost that grows
+// with the tokens and the stages of a CTA; it is taken where
+// (M + 2) * stages <= 32 (measured per layer on the LLaMA-2 7B, 13B and 70B
+// shapes, weights cold: at one token, 2 to 10 stages per CTA gain 2-15 %,
+// 28 or 32 stages lose 6-11 %; at 8 tokens 2 stages gain 6 %, 3 lose 2 %).
+// Otherwise the activation quantizer runs first, its codes and scales in
+// the caller's workspace after the GEMM's region, whose arrival counters
+// keep their fixed place at the start.
+bool fused_by_shape(int T, int M, int K, int split) {
   const int route = g_force_linear_route.load();
-  if (p.T != 16) return false;
+  if (T != 16) return false;
   if (route != 0) return route == 1;
-  const int stages = (K / 256 + p.split - 1) / p.split;     // per CTA
-  return (M <= 4 && stages <= 4) || (M <= 8 && stages <= 2);
+  const int stages = (K / 256 + split - 1) / split;         // per CTA
+  return (M + 2) * stages <= 32;
 }
+
+bool linear_fused(const Plan& p, int M, int K) { return fused_by_shape(p.T, M, K, p.split); }
 
 struct LinearLayout {
   bool fused;
@@ -743,7 +746,7 @@ int gemm_group_common(int M, int K, int gs, int bits, const int8_t* Xq, const vo
 }
 
 // A grouped linear call quantizes inside the GEMM under the same rule as a
-// single layer (16-token tiles, few stages of K per CTA, few tokens); else
+// single layer (16-token tiles, few tokens times stages of K per CTA); else
 // the activation quantizer writes codes and scales after the GEMM's region
 // of the workspace and the grouped GEMM reads them.
 struct GroupLinearLayout {
@@ -755,10 +758,7 @@ struct GroupLinearLayout {
 GroupLinearLayout group_linear_layout(int M, const int* N, int n, int K, int gs, int sms) {
   GroupLinearLayout L = {};
   L.gemm_bytes = group_gemm_bytes(M, N, n, K, gs, sms, &L.plan);
-  const int route = g_force_linear_route.load();
-  const int stages = (K / 256 + L.plan.split - 1) / L.plan.split;
-  L.fused = L.plan.T == 16 &&
-            (route != 0 ? route == 1 : ((M <= 4 && stages <= 4) || (M <= 8 && stages <= 2)));
+  L.fused = fused_by_shape(L.plan.T, M, K, L.plan.split);
   if (L.fused) {
     L.total = L.gemm_bytes;
     return L;

@@ -388,6 +388,14 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   constexpr int STAGES = Cfg::kStages;
   constexpr int ASLOTS = Cfg::kASlots;
   constexpr int NB = Cfg::kPBufs;
+  // With fused quantization the unpack warps run the quantizer's code too:
+  // the unpack loop over a stage's two weight tiles and the epilogue loop
+  // over an octet's groups stay rolled, so that the code every warp of a
+  // scheduler runs stays in its instruction cache (measured on the LLaMA-2
+  // layers: unrolled, the instruction-fetch stalls made the in-kernel
+  // quantization cost more than the separate quantizer's launch).
+  constexpr int kTileUnroll = FUSEDQ ? 1 : 2;
+  constexpr int kGroupUnroll = FUSEDQ ? 1 : 8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* xs_ring = base;                                  // STAGES * kXsBytes
@@ -715,7 +723,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
       // this row's packed bytes: tile t, chunk j at t*12288 + (j*128 + row)*16
       const uint4* src = reinterpret_cast<const uint4*>(w_ring + st.idx * Cfg::kWStageBytes) + row;
       const uint32_t col = tmem + lane_base + Cfg::kACol0 + as.idx * Cfg::kACols;
-#pragma unroll
+#pragma unroll kTileUnroll
       for (int t = 0; t < 2; ++t) {
         uint32_t w[24];
 #pragma unroll
@@ -781,7 +789,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
           __syncwarp();
         }
       }
-#pragma unroll
+#pragma unroll kGroupUnroll
       for (int gi = 0; gi < 8; ++gi) {
       const int lg = lo + gi;
       if (lg >= ngroups) break;

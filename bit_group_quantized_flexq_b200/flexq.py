@@ -287,7 +287,7 @@ def linear(x, wp, ws, N, group_size, act_bits=6, out=None, workspace_buf=None,
     """Y [M, N] FP16 of a quantized linear layer from FP16 activations x
     [M, K]: the activations are quantized to act_bits (6 or 8) by the rule of
     quantize_act, then multiplied with the packed 6-bit weights.  Batches of
-    at most 2 tokens quantize inside the GEMM (one launch; linear_launches).
+    few tokens on short K ranges quantize inside the GEMM (one launch; linear_launches).
 
     workspace_buf: a zero-filled uint8 device tensor of at least
     linear_workspace_bytes(M, N, K, gs) bytes; by default a per-device shared

@@ -145,11 +145,12 @@ def test_linear_validation_before_any_launch(L):
 
 def test_linear_workspace_layout(L):
     # small batches on short K ranges quantize inside the GEMM: the GEMM's workspace alone
-    for M, N, K in [(1, 4096, 4096), (2, 1024, 8192), (1, 384, 1024), (8, 4096, 4096)]:
+    for M, N, K in [(1, 4096, 4096), (2, 1024, 8192), (1, 384, 1024), (8, 4096, 4096),
+                    (1, 11008, 4096)]:
         assert flexq.linear_launches(M, N, K, 128) == 1
         assert flexq.linear_workspace_bytes(M, N, K, 128) == flexq.gemm_workspace_bytes(M, N, K, 128)
     # the others add the codes and the scales after the GEMM region
-    for M, N, K, gs in [(1, 11008, 4096, 128), (16, 11008, 4096, 128), (17, 4096, 4096, 128),
+    for M, N, K, gs in [(4, 11008, 4096, 128), (16, 11008, 4096, 128), (17, 4096, 4096, 128),
                         (1, 28672, 8192, 128), (256, 4096, 11008, 64), (2048, 4096, 4096, 128)]:
         assert flexq.linear_launches(M, N, K, gs) == 2
         head = max(flexq.gemm_workspace_bytes(M, N, K, gs), 4096)

@@ -1,7 +1,7 @@
 """flexq_linear_w6a6 / w6a8: a linear layer from FP16 activations.  The GEMM
 kernel can quantize the activations itself on 16-token tiles (the route the
-library takes for batches of at most 2 tokens; the tests force it at other
-sizes too), or the activation quantizer runs first.  Either way the result
+library takes for few tokens on short K ranges per CTA; the tests force it at
+other sizes too), or the activation quantizer runs first.  Either way the result
 must be bit-identical to flexq_quantize_act followed by flexq_gemm_w6a6/w6a8
 under the same plan (same codes, same scales, same arithmetic), and within
 the GEMM tolerance of the oracle's FP64 linear layer."""
@@ -208,14 +208,15 @@ def test_fused_route_stall_reports_timeout_and_context_survives(fused):
 
 
 def test_route_by_shape():
-    # one launch (quantization inside the GEMM) where each CTA streams few
-    # stages: 4096^2 splits K 8 ways (2 stages per CTA), 1024x8192 8 ways
-    # (4 stages), 11008x4096 3 ways (6 stages), 28672x8192 not at all (32)
-    for M, launches in [(1, 1), (2, 1), (3, 1), (8, 1), (9, 2), (16, 2), (17, 2), (2048, 2)]:
-        assert flexq.linear_launches(M, 4096, 4096, 128) == launches
-    for M, launches in [(1, 1), (4, 1), (5, 2)]:
-        assert flexq.linear_launches(M, 1024, 8192, 128) == launches
-    assert flexq.linear_launches(1, 11008, 4096, 128) == 2
+    # one launch (quantization inside the GEMM) where (M + 2) * stages <= 32:
+    # 4096^2 splits K 8 ways (2 stages per CTA), 1024x8192 8 ways (4
+    # stages), 11008x4096 3 ways (6 stages), 28672x8192 not at all (32)
+    for M, launches in [(1, 1), (2, 1), (8, 1), (14, 1), (15, 2), (16, 2), (17, 2), (2048, 2)]:
+        assert flexq.linear_launches(M, 4096, 4096, 128) == launches, M
+    for M, launches in [(1, 1), (6, 1), (7, 2)]:
+        assert flexq.linear_launches(M, 1024, 8192, 128) == launches, M
+    for M, launches in [(1, 1), (3, 1), (4, 2)]:
+        assert flexq.linear_launches(M, 11008, 4096, 128) == launches, M
     assert flexq.linear_launches(1, 28672, 8192, 128) == 2
     flexq.force_linear_route(1)
     assert flexq.linear_launches(16, 4096, 4096, 128) == 1
