@@ -65,10 +65,13 @@ def test_launch_count_shares_site_quantization():
     # M = 40: attn_in has 6-bit q, v and 8-bit k (2 quantizations + 3 GEMMs),
     # attn_out 2, mlp_in 1 + 2, mlp_act 2
     assert st.launches(40) == 5 + 2 + 3 + 2
-    # the 70B block at M = 1: q (8 stages per CTA) quantizes attn_in for k and
-    # v too; o, gate and down quantize first; up reuses gate's codes
+    # the 70B block at M = 1: q, k, v and o (8, 4, 4 and 8 stages per CTA)
+    # quantize inside their GEMMs; gate (32 stages) and down (28) quantize
+    # first; up reuses gate's codes
     big = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED, group_sites=False)
-    assert big.launches(1) == 2 + 1 + 1 + 2 + 2 + 1 + 2
+    assert big.launches(1) == 1 + 1 + 1 + 1 + 2 + 1 + 2
+    # at M = 4 only k and v (4 stages) still do
+    assert big.launches(4) == 2 + 1 + 1 + 2 + 2 + 1 + 2
 
 
 def test_forward_rejects_mismatched_sites():
@@ -137,9 +140,11 @@ def test_grouped_small_block_matches_grouped_calls_and_the_oracle(M):
 
 def test_grouped_70b_block_launches_and_runs():
     st = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED)
-    # q/k/v and gate/up grouped: quantizer + one grouped launch each, o and
-    # down quantizer + GEMM
-    assert st.launches(1) == 2 + 2 + 2 + 2
+    # q/k/v (11 stages per CTA) and gate/up (32) grouped: quantizer + one
+    # grouped launch each; o (8 stages) quantizes inside its GEMM; down (28)
+    # quantizer + GEMM
+    assert st.launches(1) == 2 + 1 + 2 + 2
+    assert st.launches(16) == 2 + 2 + 2 + 2
     acts = {k: v.cuda() for k, v in _acts(inputs.LLAMA2_70B_BLOCK, 16, seed=72).items()}
     out = st.forward(acts)
     assert out["k"].shape == (16, 1024) and out["up"].shape == (16, 28672)
