@@ -480,9 +480,10 @@ int gemm_common(int M, int N, int K, int gs, const int8_t* Xq, const void* Xs, c
 // dependency (about 1.5 us per layer) but adds the quantization of the
 // tile's rows to every pipeline stage of the unpack warps, a cost that grows
 // with the tokens and the stages of a CTA; it is taken where
-// (M + 2) * stages <= 32 (measured per layer on the LLaMA-2 7B, 13B and 70B
-// shapes, weights cold: at one token, 2 to 10 stages per CTA gain 2-15 %,
-// 28 or 32 stages lose 6-11 %; at 8 tokens 2 stages gain 6 %, 3 lose 2 %).
+// (M + 2) * stages <= 28 (measured per layer on the LLaMA-2 7B, 13B and 70B
+// shapes, weights cold: at one token, 2 to 8 stages per CTA gain 2-18 %, 10
+// stages lose 4 %, 28 or 32 stages 10-22 %; at 8 tokens 2 stages gain 7 %,
+// 3 lose 4 %; at 12 tokens 2 stages gain 3 %).
 // Otherwise the activation quantizer runs first, its codes and scales in
 // the caller's workspace after the GEMM's region, whose arrival counters
 // keep their fixed place at the start.
@@ -491,7 +492,7 @@ bool fused_by_shape(int T, int M, int K, int split) {
   if (T != 16) return false;
   if (route != 0) return route == 1;
   const int stages = (K / 256 + split - 1) / split;         // per CTA
-  return (M + 2) * stages <= 32;
+  return (M + 2) * stages <= 28;
 }
 
 bool linear_fused(const Plan& p, int M, int K) { return fused_by_shape(p.T, M, K, p.split); }

@@ -109,13 +109,20 @@ struct GemmCfg {
   static constexpr int kXsBytes = 2 * kXsHalf;
   static constexpr int kWStageBytes = 2 * kWTileBytes;
   static constexpr int kStageBytes = kXsBytes + kWStageBytes;
+  // activation boxes have a ring of their own, released by the MMA commit,
+  // while a weight stage is free once the unpack warps hold its bytes in
+  // registers; with more activation slots than stages (16-token tiles, whose
+  // boxes are small) a weight stage is refilled without waiting for the MMA
+  // of the stage that last used it
+  static constexpr int kXSlots = (T == 16) ? 6 : kStages;
   // scale ring: one slot holds 8 groups ("octet") of activation scales for
   // the T tokens ([8][T] fp16) and of weight scales for the 128 rows
   // ([8][128] fp16), each brought by one TMA box
   static constexpr int kScSlots = 3;
   static constexpr int kScSaBytes = 8 * T * 2;
   static constexpr int kScSlotBytes = kScSaBytes + 8 * 128 * 2;
-  static constexpr int kMainBytes = kStages * kStageBytes + kScSlots * kScSlotBytes;
+  static constexpr int kMainBytes =
+      kXSlots * kXsBytes + kStages * kWStageBytes + kScSlots * kScSlotBytes;
   // TMEM: int32 partial buffers (one per group in flight), then the A slots
   // (64 columns = 256 int8 codes per row each).  Two CTAs share an SM for
   // T <= 64, so those stay within 256 columns; T = 128 takes all 512 for
@@ -134,6 +141,7 @@ template <int T>
 struct GemmCtrl {
   uint64_t full[GemmCfg<T>::kStages];
   uint64_t empty[GemmCfg<T>::kStages];
+  uint64_t x_empty[GemmCfg<T>::kXSlots];
   uint64_t a_full[GemmCfg<T>::kASlots];
   uint64_t a_empty[GemmCfg<T>::kASlots];
   uint64_t p_full[GemmCfg<T>::kPBufs];
@@ -398,8 +406,12 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   constexpr int kGroupUnroll = FUSEDQ ? 1 : 8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* xs_ring = base;                                  // STAGES * kXsBytes
-  uint8_t* w_ring = base + STAGES * Cfg::kXsBytes;          // STAGES * 24576
+  // activation slots: the TMA's ring, or with fused quantization one slot
+  // per stage written by the unpack warps (its reuse is ordered by the A
+  // slot's release, the same MMA commit)
+  constexpr int XSL = FUSEDQ ? STAGES : Cfg::kXSlots;
+  uint8_t* xs_ring = base;                                  // kXSlots * kXsBytes
+  uint8_t* w_ring = base + Cfg::kXSlots * Cfg::kXsBytes;    // STAGES * 24576
   uint8_t* sc_ring = w_ring + STAGES * Cfg::kWStageBytes;   // kScSlots slots
   GemmCtrl<T>* ctrl = reinterpret_cast<GemmCtrl<T>*>(base + args.ctrl_offset);
   // fused quantization: per-stage activation-scale slots and their barriers
@@ -458,8 +470,9 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&ctrl->full[s], 1);
-      mbar_init(&ctrl->empty[s], 4 + 1);     // 4 unpack warps + MMA commit
+      mbar_init(&ctrl->empty[s], 4);         // 4 unpack warps (weights read)
     }
+    for (int x = 0; x < Cfg::kXSlots; ++x) mbar_init(&ctrl->x_empty[x], 1);   // MMA commit
     for (int a = 0; a < ASLOTS; ++a) {
       mbar_init(&ctrl->a_full[a], 4);        // 4 unpack warps
       mbar_init(&ctrl->a_empty[a], 1);       // MMA commit
@@ -562,7 +575,8 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         }
         if (args.stall && i == 0) continue;
         const int kb = kb0 + 2 * i;
-        uint8_t* xs = xs_ring + s * Cfg::kXsBytes;
+        const int xsl = i % XSL;
+        uint8_t* xs = xs_ring + xsl * Cfg::kXsBytes;
         if (i >= n_pre) {
           mbar_arrive_expect_tx(&ctrl->full[s], kStageTx);
           // tiles (nt, kb) and (nt, kb + 1) are adjacent in the device form
@@ -570,12 +584,21 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
                     wp + (static_cast<size_t>(nt) * KB + kb) * kWTileBytes,
                     Cfg::kWStageBytes, &ctrl->full[s]);
         }
+        // recorded before any further wait, so that a timeout below still
+        // waits (bounded) for the copy in flight
+        issued |= 1u << s;
+        parity = (parity & ~(1u << s)) | (static_cast<uint32_t>((i / STAGES) & 1) << s);
         if (!FUSEDQ) {
+          // the activation slot's previous box is free once the MMA that
+          // read it has completed
+          if (i >= XSL &&
+              !FLEXQ_WAIT(mbar_wait(&ctrl->x_empty[xsl], ((i / XSL) - 1) & 1, lim))) {
+            ok = false;
+            break;
+          }
           tma_load_2d(xs, &tmap_x, &ctrl->full[s], kb * kKBlock, mt * T);
           tma_load_2d(xs + Cfg::kXsHalf, &tmap_x, &ctrl->full[s], (kb + 1) * kKBlock, mt * T);
         }
-        issued |= 1u << s;
-        parity = (parity & ~(1u << s)) | (static_cast<uint32_t>((i / STAGES) & 1) << s);
       }
       if (!ok) record_status(args.status, kStatusTimeout, 0);
       FLEXQ_ROLE_DONE(0, nst);
@@ -611,7 +634,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
         constexpr int SPG = GS / 32;                     // MMAs per group
         constexpr bool kBatch = NB >= 2 * G;
         constexpr uint32_t idesc = idesc_i8(kTileRows, T);
-        RingPos<STAGES> st;
+        RingPos<XSL> xp;
         RingPos<ASLOTS> as;
         RingPos<NB> pb;                                  // buffer of the next group
         for (int i = 0; i < nst; ++i) {
@@ -627,7 +650,7 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
           }
           tc_fence_after();
           const uint32_t a_col = tmem + Cfg::kACol0 + as.idx * Cfg::kACols;
-          const uint64_t b_desc = desc0 + ((st.idx * Cfg::kXsBytes) >> 4);
+          const uint64_t b_desc = desc0 + ((xp.idx * Cfg::kXsBytes) >> 4);
 #pragma unroll
           for (int j = 0; j < G; ++j) {
             if constexpr (!kBatch) {
@@ -648,9 +671,9 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
             mma_commit(&ctrl->p_full[pb.idx]);
             pb.next();
           }
-          mma_commit(&ctrl->empty[st.idx]);     // frees the smem stage
+          if (!FUSEDQ) mma_commit(&ctrl->x_empty[xp.idx]);   // frees the activation slot
           mma_commit(&ctrl->a_empty[as.idx]);   // frees the A slot
-          st.next();
+          xp.next();
           as.next();
         }
         return true;

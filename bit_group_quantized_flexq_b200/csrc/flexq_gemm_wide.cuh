@@ -49,6 +49,7 @@ namespace flexq {
 
 struct WideCfg {
   static constexpr int T = 128;                       // tokens per tile (MMA N)
+  static constexpr int kBandN = 32;                   // weight tiles per raster band
   static constexpr int kThreads = 512;
   static constexpr int kStages = 3;
   static constexpr int kKStage = 2 * kKBlock;         // codes of K per stage
@@ -154,9 +155,21 @@ __global__ void __launch_bounds__(WideCfg::kThreads, 1)
     ks = u - (u / args.split) * args.split;
     S = args.split;
   }
-  const int nt = tile % args.tiles_n;
-  const int mt = tile / args.tiles_n;
   const int M = args.M, N = args.N, K = args.K, gs = args.gs;
+  // output tile -> (weight tile nt, token tile mt) in bands of kBandN weight
+  // tiles: inside a band the weight tile varies fastest and every token tile
+  // passes the band's weight rows, so the CTAs in flight share a few weight
+  // strips, which stay in L2 while the band lasts, and the packed weights are
+  // read from DRAM about once (the activations once per band) instead of once
+  // per token tile.
+  const int tiles_m = (M + T - 1) / T;
+  constexpr int kBandN = Cfg::kBandN;
+  const int band = tile / (kBandN * tiles_m);
+  const int n_band0 = band * kBandN;
+  const int band_n = min(kBandN, args.tiles_n - n_band0);
+  const int in_band = tile - band * kBandN * tiles_m;
+  const int nt = n_band0 + in_band % band_n;
+  const int mt = in_band / band_n;
   const int KB = K / kKBlock;
   const int units = K / Cfg::kKStage;
   const int u0 = static_cast<int>((static_cast<long long>(ks) * units) / S);

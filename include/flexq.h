@@ -203,7 +203,7 @@ size_t flexq_linear_workspace_bytes(int M, int N, int K, int group_size);
  * flexq_linear_launches -- kernel launches of one linear call for a shape:
  * 1 where the activations are quantized inside the GEMM, 2 otherwise
  * (quantizer, GEMM).  The GEMM quantizes on 16-token tiles where
- * (M + 2) * stages <= 32, stages being the stages of 256 codes of K that each
+ * (M + 2) * stages <= 28, stages being the stages of 256 codes of K that each
  * CTA streams (where that is faster than a separate quantizer).
  * 0 for unsupported shapes and M <= 0.  Pure host computation.
  */
