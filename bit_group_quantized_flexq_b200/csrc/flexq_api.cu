@@ -893,6 +893,28 @@ int flexq_quantize_weight_layout(int N, int K, int group_size, int layout, const
   return ok();
 }
 
+int flexq_debug_export_canonical(int N, int K, int layout, const void* Wq_packed,
+                                 void* W_canonical, void* stream) {
+  if (layout != FLEXQ_LAYOUT_BYTE_ALIGNED && layout != FLEXQ_LAYOUT_4_2)
+    return fail(FLEXQ_ERR_INVALID_ARG, "layout=%d is not a weight layout", layout);
+  int rc = check_gemm_shape(1, N, K, 128);
+  if (rc) return rc;
+  const void* ptrs[] = {Wq_packed, W_canonical};
+  const char* names[] = {"Wq_packed", "W_canonical"};
+  if ((rc = check_ptrs(2, ptrs, names))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const dim3 grid(static_cast<unsigned>(K / 128), static_cast<unsigned>(N / 128));
+  const uint8_t* wp = static_cast<const uint8_t*>(Wq_packed);
+  uint8_t* out = static_cast<uint8_t*>(W_canonical);
+  if (layout == FLEXQ_LAYOUT_4_2)
+    flexq::export_canonical_kernel<1><<<grid, flexq::kTileRows, 0, s>>>(wp, out, K);
+  else
+    flexq::export_canonical_kernel<0><<<grid, flexq::kTileRows, 0, s>>>(wp, out, K);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "export_canonical_kernel launch");
+  return ok();
+}
+
 int flexq_quantize_act(int M, int K, int group_size, int bits, const void* X_fp16, int8_t* Xq,
                        void* X_scales_fp16, void* stream) {
   if (M < 0 || K <= 0) return fail(FLEXQ_ERR_INVALID_ARG, "sizes must be M >= 0, K > 0 (M=%d K=%d)", M, K);

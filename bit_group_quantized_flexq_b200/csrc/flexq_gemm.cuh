@@ -281,6 +281,48 @@ __device__ __forceinline__ void unpack_row_tile(const uint32_t (&w)[24], uint32_
   }
 }
 
+// The device form of packed weights (either layout) -> the canonical form:
+// row-major, codes 4j .. 4j+3 of a row as the 24-bit word
+// u0 | u1 << 6 | u2 << 12 | u3 << 18 (u_i = code_i & 0x3F) in bytes 3j .. 3j+2,
+// little endian.  One thread per weight row of a 128 x 128 tile: it reads the
+// row's six 16-byte chunks, unpacks them as the GEMM does (code * 4 per byte)
+// and writes the row's 96 canonical bytes of the tile.
+template <int LAYOUT>
+__global__ void __launch_bounds__(kTileRows) export_canonical_kernel(
+    const uint8_t* __restrict__ wp, uint8_t* __restrict__ out, int K) {
+  const int kb = blockIdx.x, nt = blockIdx.y, r = threadIdx.x;
+  const int KB = K / kKBlock;
+  const uint4* tile =
+      reinterpret_cast<const uint4*>(wp + (static_cast<size_t>(nt) * KB + kb) * kWTileBytes);
+  uint32_t w[24];
+#pragma unroll
+  for (int j = 0; j < 6; ++j) {
+    const uint4 v = __ldg(tile + j * kTileRows + r);
+    w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+  }
+  uint32_t c[32];
+  unpack_row_tile<LAYOUT>(w, c);
+  uint32_t o[24];
+#pragma unroll
+  for (int q4 = 0; q4 < 8; ++q4) {
+    uint32_t t[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t v = c[4 * q4 + i];                // four codes * 4, one per byte
+      t[i] = ((v >> 2) & 0x3Fu) | (((v >> 10) & 0x3Fu) << 6) | (((v >> 18) & 0x3Fu) << 12) |
+             (((v >> 26) & 0x3Fu) << 18);
+    }
+    o[3 * q4] = t[0] | (t[1] << 24);
+    o[3 * q4 + 1] = (t[1] >> 8) | (t[2] << 16);
+    o[3 * q4 + 2] = (t[2] >> 16) | (t[3] << 8);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(nt) * kTileRows + r) *
+                                                  (static_cast<size_t>(K) * 3 / 4) +
+                                        static_cast<size_t>(kb) * 96);
+#pragma unroll
+  for (int j = 0; j < 6; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+}
+
 // ---------------------------------------------------------------------------
 // Fused activation quantization (FUSEDQ, token tiles of 16 rows): the kernel
 // reads the FP16 activations itself.  At stage i unpack warp q quantizes rows

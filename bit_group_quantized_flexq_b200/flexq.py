@@ -82,6 +82,7 @@ def lib():
                                         ctypes.POINTER(c_int)]),
             "flexq_debug_force_plan": (c_int, [c_int, c_int]),
             "flexq_linear_launches": (c_int, [c_int, c_int, c_int, c_int]),
+            "flexq_debug_export_canonical": (c_int, [c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
             "flexq_debug_force_linear_route": (c_int, [c_int]),
             "flexq_set_wait_limit_ns": (c_int, [ctypes.c_uint64]),
             "flexq_debug_inject_stall": (c_int, [c_int]),
@@ -352,6 +353,17 @@ def debug_group_partials(xq, wp, N, group_size, out=None):
     _need(out, "out", torch.int32, (G, M, N))
     _check(lib().flexq_debug_group_partials(M, N, K, group_size, _ptr(xq), _ptr(wp), _ptr(out),
                                             _stream(xq)))
+    return out
+
+
+def export_canonical(wp, N, K, layout=LAYOUT_BYTE_ALIGNED, out=None):
+    """The packed weights wp (device form of `layout`) in the canonical 6-bit
+    form: uint8 [N, 3K/4], four codes per three bytes, row-major."""
+    _need(wp, "packed", torch.uint8, (N * K * 3 // 4,))
+    if out is None:
+        out = torch.empty(N, K * 3 // 4, dtype=torch.uint8, device=wp.device)
+    _need(out, "out", torch.uint8, (N, K * 3 // 4))
+    _check(lib().flexq_debug_export_canonical(N, K, layout, _ptr(wp), _ptr(out), _stream(wp)))
     return out
 
 

@@ -390,6 +390,25 @@ int flexq_debug_group_partials(int M, int N, int K, int group_size,
                                int32_t* P, void* stream);
 
 /*
+ * flexq_debug_export_canonical -- the packed weights in the canonical 6-bit
+ * form, for tests and for interchange with other tools.  Passage: uniform
+ * 6-bit weights stored four codes to three bytes (arXiv abstract; blog,
+ * "Bridging Software and Hardware with BTC").
+ *   layout       FLEXQ_LAYOUT_BYTE_ALIGNED or FLEXQ_LAYOUT_4_2: the form of
+ *                Wq_packed (as written by flexq_quantize_weight_layout).
+ *   Wq_packed    in, device, flexq_weight_packed_bytes(N, K, 128) bytes.
+ *   W_canonical  out, device, 3*N*K/4 bytes, row-major: for codes c0..c3 at
+ *                k = 4j..4j+3 of row n (u_i = c_i & 63) the 24-bit word
+ *                u0 | u1<<6 | u2<<12 | u3<<18, little endian, at bytes
+ *                n*(3K/4) + 3j .. +2.  Owned by the caller.
+ * Shapes as for the GEMM (N % 128 == 0, K % 256 == 0); both pointers 16-byte
+ * aligned (FLEXQ_ERR_MISALIGNED), checked before anything is enqueued.
+ * Asynchronous on `stream`.
+ */
+int flexq_debug_export_canonical(int N, int K, int layout, const void* Wq_packed,
+                                 void* W_canonical, void* stream);
+
+/*
  * flexq_gemm_plan -- the launch the GEMM entry points would use for a shape
  * given enough workspace: tokens per tile (16, 32, 64 or 128), K-split factor
  * (CTAs that share an output tile, each over its own range of K) and the

@@ -228,3 +228,15 @@ def test_layout_validation_before_any_launch(L):
     assert f(4, 256, 256, 128, 6, -1, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == \
         flexq.FLEXQ_ERR_INVALID_ARG
     assert f(0, 256, 256, 128, 6, 1, FAKE, FAKE, FAKE, FAKE, NULL, 0, NULL) == flexq.FLEXQ_OK
+
+
+def test_export_canonical_validation_before_any_launch(L):
+    f = L.flexq_debug_export_canonical
+    assert f(256, 512, 2, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_INVALID_ARG          # layout
+    assert f(200, 512, 0, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED          # N % 128
+    assert f(256, 384, 1, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_UNSUPPORTED          # K % 256
+    assert f(0, 512, 0, FAKE, FAKE, NULL) == flexq.FLEXQ_ERR_INVALID_ARG            # N <= 0
+    assert f(256, 512, 0, NULL, FAKE, NULL) == flexq.FLEXQ_ERR_INVALID_ARG
+    assert b"Wq_packed" in L.flexq_last_error_message()
+    assert f(256, 512, 0, FAKE, MISALIGNED, NULL) == flexq.FLEXQ_ERR_MISALIGNED
+    assert b"W_canonical" in L.flexq_last_error_message()
