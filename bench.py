@@ -35,6 +35,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -251,17 +252,24 @@ def kernel_source_digest():
     return h.hexdigest()[:16]
 
 
+TRAFFIC_SUMMARY = os.path.join("profiles", "gemm_w6ax_wide_70b_step_traffic.md")
+
+
 def profiled_traffic():
     """DRAM bytes per launch of the dominant GEMM from the committed ncu
-    summary, or None when the kernel source changed since that capture."""
-    p = os.path.join(ROOT, "profiles", "gemm_wide_traffic.json")
+    summary of the bench step's wide launches (its `dram_bytes_per_launch`
+    and `kernel_src_sha` lines), or None when that summary is missing or the
+    kernel sources changed since the capture."""
+    p = os.path.join(ROOT, TRAFFIC_SUMMARY)
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        d = json.load(f)
-    if d.get("kernel_src_sha") != kernel_source_digest():
+        text = f.read()
+    sha = re.search(r"kernel_src_sha:\s*([0-9a-f]+)", text)
+    nbytes = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not sha or not nbytes or sha.group(1) != kernel_source_digest():
         return None
-    return d.get("dram_bytes_per_launch")
+    return int(nbytes.group(1))
 
 
 # ------------------------------------------------------------ flexq arm ----
