@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("gs", [32, 64, 128, 256])
 @pytest.mark.parametrize("bits", [6, 8])
-@pytest.mark.parametrize("M,K", [(1, 256), (3, 512), (17, 1024), (130, 768)])
+@pytest.mark.parametrize("M,K", [(1, 256), (3, 512), (9, 2304), (16, 8192), (17, 1024), (130, 768)])
 def test_act_quant_bit_exact(M, K, gs, bits):
     if K % gs:
         pytest.skip("K must be a multiple of the group size")
