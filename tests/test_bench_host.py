@@ -97,3 +97,20 @@ def test_headline_workload_is_the_llama2_70b_configuration():
     # gate and up read the same input; every other layer its own
     assert len({site for (*_, site) in layers}) == 4
     assert "LLaMA-2-70B" in bench.workload_name(ms, layers)
+
+
+def test_profiled_traffic_follows_the_kernel_source_digest(tmp_path, monkeypatch):
+    # the committed summary carries the digest of the sources it was captured
+    # with; the bench reports its byte count only while they still match
+    text = open(os.path.join(bench.ROOT, bench.TRAFFIC_SUMMARY)).read()
+    assert "kernel_src_sha:" in text and "dram_bytes_per_launch:" in text
+    root = tmp_path / "repo"
+    (root / "profiles").mkdir(parents=True)
+    summary = root / bench.TRAFFIC_SUMMARY
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    monkeypatch.setattr(bench, "kernel_source_digest", lambda: "00c0ffee")
+    assert bench.profiled_traffic() is None                       # no summary
+    summary.write_text("kernel_src_sha: 00c0ffee\ndram_bytes_per_launch: 12345\n")
+    assert bench.profiled_traffic() == 12345
+    summary.write_text("kernel_src_sha: deadbeef\ndram_bytes_per_launch: 12345\n")
+    assert bench.profiled_traffic() is None                       # sources changed
