@@ -697,41 +697,60 @@ def stack_diagnostics(device, hbm_gbs, int8_peak_tops, ms=(1, 16)):
     it: the layers of one input site as one grouped launch, each with its
     own packed weights (`by_m`, the default); every layer its own launch
     (`by_m_single_launches`); the layers of a site merged into one weight
-    matrix (`by_m_fused_sites`, a different weight layout)."""
+    matrix (`by_m_fused_sites`, a different weight layout).  The same for
+    the LLaMA-2-7B block, W6A6 (`llama2_7b_block`; two copies of the block
+    run in turn, 311 MB of packed weights, so that they do not sit in L2)."""
     import torch
     from bit_group_quantized_flexq_b200 import inputs, stack
     res = {}
     for key, kw in (("by_m", {}), ("by_m_single_launches", {"group_sites": False}),
                     ("by_m_fused_sites", {"fuse_sites": True})):
         st = stack.LayerStack(inputs.LLAMA2_70B_BLOCK, stack.LLAMA2_70B_MIXED, device=device, **kw)
-        res[key] = _stack_rows(st, device, hbm_gbs, int8_peak_tops, ms)
+        res[key] = _stack_rows([st], device, hbm_gbs, int8_peak_tops, ms)
         bits, gs, packed = st.bits, st.gs, st.packed_bytes()
         del st
         torch.cuda.empty_cache()
+    cfg7 = {"group_size": 128, "act_bits": {name: 6 for name, _, _, _ in inputs.LLAMA2_7B_BLOCK}}
+    res7 = {}
+    for key, kw in (("by_m", {}), ("by_m_single_launches", {"group_sites": False})):
+        sts = [stack.LayerStack(inputs.LLAMA2_7B_BLOCK, cfg7, device=device, seed=c, **kw)
+               for c in range(2)]
+        res7[key] = _stack_rows(sts, device, hbm_gbs, int8_peak_tops, ms)
+        del sts
+        torch.cuda.empty_cache()
     return {"block": "LLaMA-2-70B (q, k, v, o, gate, up, down)",
-            "act_bits": bits, "group_size": gs, "packed_MB": round(packed / 1e6, 1), **res}
+            "act_bits": bits, "group_size": gs, "packed_MB": round(packed / 1e6, 1), **res,
+            "llama2_7b_block": {"act_bits": 6, "group_size": 128, "copies": 2, **res7}}
 
 
-def _stack_rows(st, device, hbm_gbs, int8_peak_tops, ms):
+def _stack_rows(stacks, device, hbm_gbs, int8_peak_tops, ms):
+    """Per M, one forward of every stack in `stacks` in turn (each its own
+    weights) per timed pass; figures for the whole pass."""
     import torch
     from bit_group_quantized_flexq_b200 import inputs
     stream = torch.cuda.Stream(device)
     rows = []
+    st0 = stacks[0]
     for M in ms:
         acts = {site: inputs.activations(M, K, outlier_frac=0.005, outlier_scale=50.0,
                                          seed=inputs.layer_seed("70b-x", M, site)).to(device)
-                for site, K in st.sites().items()}
+                for site, K in st0.sites().items()}
         out = {name: torch.empty(M, N, dtype=torch.float16, device=device)
-               for name, N, K, _ in st.layers}
+               for name, N, K, _ in st0.layers}
+
+        def passes():
+            for st in stacks:
+                st.forward(acts, out)
         reps = 2 if M >= 4096 else 5
-        us = _graph_time_us(lambda: st.forward(acts, out), device, stream, reps)
-        flops = sum(2.0 * M * N * K for _, N, K, _ in st.layers)
-        nbytes = sum(linear_bytes(M, N, K, st.gs) for _, N, K, _ in st.layers)
+        us = _graph_time_us(passes, device, stream, reps)
+        flops = len(stacks) * sum(2.0 * M * N * K for _, N, K, _ in st0.layers)
+        nbytes = len(stacks) * sum(linear_bytes(M, N, K, st0.gs) for _, N, K, _ in st0.layers)
         gbs = nbytes / (us * 1e-6) / 1e9
         tops = flops / (us * 1e-6) / 1e12
         bound, frac = roofline(flops, nbytes, us, hbm_gbs, int8_peak_tops)
         rows.append({"M": M, "us": round(us, 2), "TOPS": round(tops, 2), "GB/s": round(gbs, 1),
-                     "bound": bound, "frac": round(frac, 4), "launches": st.launches(M)})
+                     "bound": bound, "frac": round(frac, 4),
+                     "launches": len(stacks) * st0.launches(M)})
         del acts, out
     return rows
 

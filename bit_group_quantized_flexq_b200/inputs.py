@@ -28,6 +28,14 @@ LLAMA2_7B_LAYERS = [
     ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008),
 ]
 LLAMA2_7B_M = [1, 16, 256, 2048]
+# One LLaMA-2-7B transformer block with the input site of each layer (as
+# LLAMA2_70B_BLOCK below).
+LLAMA2_7B_BLOCK = [
+    ("q", 4096, 4096, "attn_in"), ("k", 4096, 4096, "attn_in"), ("v", 4096, 4096, "attn_in"),
+    ("o", 4096, 4096, "attn_out"),
+    ("gate", 11008, 4096, "mlp_in"), ("up", 11008, 4096, "mlp_in"),
+    ("down", 4096, 11008, "mlp_act"),
+]
 
 LLAMA2_13B_LAYERS = [("qkvo", 5120, 5120), ("gate_up", 13824, 5120),
                      ("down", 5120, 13824)]
