@@ -973,15 +973,11 @@ __global__ void __launch_bounds__(GemmCfg<T>::kThreads, GemmCfg<T>::kMinBlocks)
     FLEXQ_CTA_TIME(6);
     if (threadIdx.x == 0) {
       // the barrier orders the CTA's partial stores before this thread's
-      // fence, which releases them with the count; the last CTA's fence
-      // acquires the other CTAs' partials before the barrier below
-      __threadfence();
-      const unsigned old = atomicAdd(&args.ws_cnt[st_idx], 1u);
+      // acquire-release add, which releases them with the count; the last
+      // CTA's add acquires the other CTAs' partials before the barrier below
+      const unsigned old = atom_add_acq_rel_gpu(&args.ws_cnt[st_idx], 1u);
       const bool last = old == static_cast<unsigned>(S - 1);
-      if (last) {
-        args.ws_cnt[st_idx] = 0u;
-        __threadfence();
-      }
+      if (last) args.ws_cnt[st_idx] = 0u;    // for the next launch (ordered by the kernel boundary)
       ctrl->is_last = last ? 1u : 0u;
     }
     __syncthreads();

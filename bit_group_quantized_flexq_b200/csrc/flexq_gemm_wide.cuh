@@ -234,17 +234,13 @@ __global__ void __launch_bounds__(WideCfg::kThreads, 1)
     if (!PARTIALS && S > 1) {
       named_bar_sync(2, Cfg::kThreads);
       if (threadIdx.x == 0) {
-        // the barrier orders the CTA's partial stores before this fence,
-        // which releases them with the count; the last CTA's fence acquires
-        // the other CTAs' partial tiles before barrier 3
-        __threadfence();
+        // the barrier orders the CTA's partial stores before this
+        // acquire-release add, which releases them with the count; the last
+        // CTA's add acquires the other CTAs' partial tiles before barrier 3
         const size_t st_idx = static_cast<size_t>(tile - args.n_full);
-        const unsigned old = atomicAdd(&args.ws_cnt[st_idx], 1u);
+        const unsigned old = atom_add_acq_rel_gpu(&args.ws_cnt[st_idx], 1u);
         const bool last = old == static_cast<unsigned>(S - 1);
-        if (last) {
-          args.ws_cnt[st_idx] = 0u;
-          __threadfence();
-        }
+        if (last) args.ws_cnt[st_idx] = 0u;  // for the next launch (ordered by the kernel boundary)
         ctrl->is_last = last ? 1u : 0u;
       }
       named_bar_sync(3, Cfg::kThreads);

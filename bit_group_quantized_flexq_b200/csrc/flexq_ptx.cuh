@@ -155,6 +155,15 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 
 // Orders this thread's generic-proxy writes to shared memory before later
 // async-proxy reads of it (a tensor-core operand the thread stored itself).
+// Atomic add at GPU scope with acquire-release semantics: releases the
+// writes this thread has observed (cumulatively, e.g. through a CTA barrier)
+// and acquires those released by earlier adders.  Returns the old value.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
