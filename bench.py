@@ -908,7 +908,40 @@ def int8_library_context(W, device, M, reps=20):
         return {"unavailable": str(exc).splitlines()[0][:200]}
 
 
+def gpu_local_cpus(index):
+    """The host CPUs NVML reports as local to GPU `index` (its NUMA node), or
+    None when NVML cannot tell."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByIndex(index)
+        ncpu = os.cpu_count() or 1
+        words = pynvml.nvmlDeviceGetCpuAffinity(h, (ncpu + 63) // 64)
+        cpus = {64 * w + b for w, mask in enumerate(words) for b in range(64) if (mask >> b) & 1}
+        return cpus or None
+    except Exception:
+        return None
+
+
 def run_e2e(W, args, device, world):
+    """Pins this process to the GPU's local CPUs while the host buffers are
+    allocated and the copies run (so the pinned pages sit on the GPU's NUMA
+    node), then restores the previous affinity."""
+    saved = os.sched_getaffinity(0)
+    local = gpu_local_cpus(device.index if device.index is not None else 0)
+    pinned = sorted(local & saved) if local else []
+    if pinned:
+        os.sched_setaffinity(0, pinned)
+    try:
+        res = _run_e2e(W, args, device, world)
+    finally:
+        os.sched_setaffinity(0, saved)
+    res["host_cpus"] = (f"{len(pinned)} CPUs local to the GPU (NVML)" if pinned
+                        else "unpinned (NVML gave no CPU affinity)")
+    return res
+
+
+def _run_e2e(W, args, device, world):
     """The same metric through the public API with host buffers: every step
     copies each layer's FP16 input from pinned host memory and each output
     back to pinned host memory.  Copies in, layer calls and copies out run
