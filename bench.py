@@ -245,10 +245,15 @@ def measured_peaks():
 
 
 def kernel_source_digest():
+    """Digest of the GEMM sources' code: comments and whitespace removed, so
+    that only a change of the code itself marks a profiled figure stale."""
     h = hashlib.sha256()
     for f in ("flexq_gemm.cuh", "flexq_gemm_wide.cuh", "flexq_ptx.cuh", "flexq_api.cu"):
-        with open(os.path.join(ROOT, "bit_group_quantized_flexq_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "bit_group_quantized_flexq_b200", "csrc", f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

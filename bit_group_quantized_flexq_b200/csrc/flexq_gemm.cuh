@@ -19,11 +19,13 @@
 // tiles).
 //
 // Warp roles (all pipeline waits are bounded, see mbar_wait):
-//   warp 0      producer: per stage, two TMA boxes of the int8 activations
-//               (T rows x 128 B each, 128-byte swizzle) and one 24576-byte
-//               bulk copy of two consecutive packed weight tiles into a
-//               STAGES-deep shared-memory ring; per 8 groups, the group
-//               scales;
+//   warp 0      producer: per stage, one 24576-byte bulk copy of two
+//               consecutive packed weight tiles into a STAGES-deep weight
+//               ring (a stage is free again once the unpack warps hold its
+//               bytes) and two TMA boxes of the int8 activations (T rows x
+//               128 B each, 128-byte swizzle) into an activation ring of
+//               kXSlots slots (free again after the MMAs that read it); per
+//               8 groups, the group scales;
 //   warp 1      TMEM allocator and MMA issuer: 8 MMAs (K = 32 each) per
 //               stage into the int32 partial buffer of the current group
 //               (kPBufs buffers of T columns), one commit per group;
